@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""TPLA decode benchmark: one JSON line on rank 0.
+
+A step is the whole decode hot path for one batch: tpla_append_kv of one new
+token per sequence (Hadamard reparameterisation + sliced RMSNorm), then the
+split-KV attention and the combine (split merge, W_UV, shard sum).  The
+default workload is the DeepSeek-V3 attention shape at TP degree g = 2, one
+rank's share (tpla_decode_shard, shard 0), batch 16, 32768 cached tokens per
+sequence; every input is seeded synthetic data resident in HBM.  The
+per-shard cache (335 MB) is larger than the 126 MB L2, so no L2 flush is
+needed between steps.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+Under torchrun (N > 1) every rank runs an independent replica (the path has
+no exchange step on one node here); the reported time is the max over ranks.
+"""
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "TPLA decode µs/step and latent-cache GB/s (% of B200 HBM peak) at 32K ctx"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------- workload description
+
+def workload_spec(name):
+    from latent_attention_decode_tpla_b200 import inputs as gen
+    spec = dict(gen.WORKLOADS[name])
+    spec["name"] = name
+    spec.setdefault("mode", "shard" if spec["g"] > 1 else "full")
+    return spec
+
+
+def algorithmic_bytes(spec, seq_lens_sum, mode):
+    """Bytes the attention stage must read: cache rows (+ queries).  Per shard call: latent slice
+    plus RoPE key per token; all shards: the whole latent plus one RoPE key per token."""
+    L, R, g, H, B = spec["L"], spec["R"], spec["g"], spec["H"], spec["B"]
+    cols = (L // g + R) if mode == "shard" else (L + R)
+    cache = seq_lens_sum * cols * 2
+    queries = B * H * cols * 2
+    return cache, cache + queries
+
+
+def source_digest():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "latent_attention_decode_tpla_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """dram bytes per launch from the committed ncu summary, if it was taken on the current sources."""
+    path = os.path.join(ROOT, "profiles", "%s_%s.txt" % (kernel, workload))
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for ln in open(path):
+        if ":" in ln:
+            k, v = ln.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_digest") != source_digest():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        try:
+            return json.load(open(path)), "measured"
+        except ValueError:
+            pass
+    return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+# ---------------------------------------------------------------- clocks sampling
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) == 7:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm = []
+        mx = []
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[0]))
+                mx.append(float(r[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_init():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world, local
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(x):
+    """Max of a float over ranks (a host-side timing reduction, not a data-path collective)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x):
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def build_device_workload(spec, seed=0):
+    """Seeded synthetic inputs created on the current GPU (bf16 cache N(0,1): unit RMS per shard row)."""
+    import torch
+    from latent_attention_decode_tpla_b200 import inputs as gen
+    from latent_attention_decode_tpla_b200 import tpla
+    B, H, L, R, dv, g = spec["B"], spec["H"], spec["L"], spec["R"], spec["dv"], spec["g"]
+    lens = gen.workload_seq_lens(spec, seed)
+    maxp = gen.pages_for(int(lens.max()))
+    num_pages = B * maxp
+    gd = torch.Generator(device="cuda")
+    gd.manual_seed(1000 * seed + 77)
+
+    def rn(*shape, std=1.0):
+        return (torch.randn(*shape, generator=gd, device="cuda", dtype=torch.float32) * std).to(torch.bfloat16)
+
+    w = {}
+    w["ckv"] = torch.empty((num_pages, g, 64, L // g), dtype=torch.bfloat16, device="cuda")
+    step = max(1, (1 << 27) // (g * 64 * (L // g)))
+    for i in range(0, num_pages, step):
+        j = min(num_pages, i + step)
+        w["ckv"][i:j] = rn(j - i, g, 64, L // g)
+    w["kpe"] = rn(num_pages, 64, R)
+    w["q"] = rn(B, H, L)
+    w["q_pe"] = rn(B, H, R)
+    w["w_uv"] = rn(H, L, dv, std=1.0 / math.sqrt(L))
+    w["x_new"] = rn(B, L)
+    w["kpe_new"] = rn(B, R)
+    w["block_table"] = gen.block_table(B, maxp, num_pages, seed).cuda()
+    w["seq_lens"] = lens.cuda()
+    w["positions"] = (lens - 1).clamp(min=0).cuda()      # the step's token is the newest cached one
+    dims = tpla.make_dims(B=B, H=H, L=L, R=R, dv=dv, g=g, max_pages_per_seq=maxp, num_pages=num_pages,
+                          softmax_scale=gen.softmax_scale(spec))
+    w["dims"] = dims
+    w["workspace"] = tpla.alloc_workspace(dims)
+    w["out"] = torch.empty((B, H, dv), dtype=torch.float32, device="cuda")
+    w["lens_sum"] = int(lens.sum())
+    return w
+
+
+def gpu_step(w, spec, ev_attn=None):
+    from latent_attention_decode_tpla_b200 import tpla
+    shard = 0 if spec["mode"] == "shard" else -1
+    d = w["dims"]
+    tpla.append_kv(d, w["x_new"], w["kpe_new"], spec["transform"], w.get("R_dense"), None, 1e-6,
+                   w["positions"], w["block_table"], w["ckv"], w["kpe"])
+    if ev_attn is not None:
+        ev_attn[0].record()
+    tpla.attention(d, shard, w["q"], w["q_pe"], w["ckv"], w["kpe"], w["block_table"], w["seq_lens"],
+                   w["workspace"])
+    if ev_attn is not None:
+        ev_attn[1].record()
+    tpla.combine(d, shard, w["seq_lens"], w["w_uv"], w["out"], w["workspace"])
+
+
+def run_gpu_arm(args, spec, rank, world, local):
+    import torch
+    from latent_attention_decode_tpla_b200 import inputs as gen
+    from latent_attention_decode_tpla_b200 import tpla
+    torch.cuda.set_device(local)
+    w = build_device_workload(spec, seed=0)
+    if spec["transform"] == 2:
+        w["R_dense"] = gen.random_orthogonal(spec["L"], 0).cuda()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        gpu_step(w, spec)
+    torch.cuda.synchronize()
+    st = tpla.check_device_status()
+    if st != tpla.TPLA_OK:
+        raise RuntimeError("device status after warm-up: " + tpla.status_string(st))
+
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(K):
+        gpu_step(w, spec, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier()
+    ms = start.elapsed_time(end) / K
+    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    ms_max = max_over_ranks(ms)
+    attn_ms_max = max_over_ranks(attn_ms)
+
+    # end to end through the public API with host buffers: H2D of the step's inputs (pinned),
+    # the step, D2H of the result, read on the host every step
+    host = {k: w[k].cpu().pin_memory() for k in ("q", "q_pe", "x_new", "kpe_new")}
+    out_host = torch.empty(w["out"].shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    done = torch.cuda.Event()
+    torch.cuda.synchronize()
+    barrier()
+    e_start.record(stream)
+    for _ in range(K):
+        for k, t in host.items():
+            w[k].copy_(t, non_blocking=True)
+        gpu_step(w, spec)
+        out_host.copy_(w["out"], non_blocking=True)
+        done.record(stream)
+        done.synchronize()
+        _ = float(out_host[0, 0, 0])
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / K)
+    st = tpla.check_device_status()
+    if st != tpla.TPLA_OK:
+        raise RuntimeError("device status after timing: " + tpla.status_string(st))
+
+    kernel = tpla.get_option(tpla.OPT_LAST_ATTENTION_KERNEL)
+    cache_b, attn_b = algorithmic_bytes(spec, w["lens_sum"], spec["mode"])
+    total_cache = sum_over_ranks(cache_b)
+    return dict(ms=ms_max, attn_ms=attn_ms_max, e2e_ms=e2e_ms, cache_bytes=cache_b, attn_bytes=attn_b,
+                total_cache=total_cache, clocks=clocks, h2d=h2d, d2h=d2h, launches=3 * K, kernel=kernel,
+                lens_sum=w["lens_sum"])
+
+
+# ---------------------------------------------------------------- oracle (CPU) arm
+
+def oracle_sample(spec, seed=0, T=None):
+    """One sequence of the workload (shard 0 for per-shard workloads) as CPU float64 arrays."""
+    import numpy as np
+    import torch
+    from latent_attention_decode_tpla_b200 import inputs as gen
+    lens = gen.workload_seq_lens(spec, seed)
+    T = int(lens.max()) if T is None else T
+    d = gen.make_workload(B=1, H=spec["H"], L=spec["L"], R=spec["R"], dv=spec["dv"], g=spec["g"], seq_lens=[T],
+                          seed=seed, extra_pages=0)
+    f = lambda t: t.to(torch.float64).numpy()
+    s = dict(q=f(d["q"]), q_pe=f(d["q_pe"]), ckv=f(d["ckv"]), kpe=f(d["kpe"]), bt=d["block_table"].numpy(),
+             w_uv=f(d["w_uv"]), x_new=f(d["x_new"]), kpe_new=f(d["kpe_new"]), T=T,
+             maxp=d["max_pages_per_seq"])
+    if spec["transform"] == 2:
+        s["R_dense"] = gen.random_orthogonal(spec["L"], seed).numpy().astype(np.float64)
+    return s
+
+
+def oracle_step(spec, s):
+    """The oracle's version of one step on the sample: append one token, then decode."""
+    from latent_attention_decode_tpla_b200 import inputs as gen
+    from oracle import tpla_ref as ref
+    scale = gen.softmax_scale(spec)
+    ref.append_kv(s["x_new"], s["kpe_new"], [s["T"] - 1], s["bt"], s["ckv"], s["kpe"], g=spec["g"],
+                  max_pages_per_seq=s["maxp"], transform=spec["transform"], R_dense=s.get("R_dense"), eps=1e-6)
+    if spec["mode"] == "shard":
+        return ref.decode_shard(s["q"], s["q_pe"], s["ckv"], s["kpe"], s["bt"], [s["T"]], scale, 0,
+                                max_pages_per_seq=s["maxp"], w_uv=s["w_uv"])
+    return ref.decode(s["q"], s["q_pe"], s["ckv"], s["kpe"], s["bt"], [s["T"]], scale,
+                      max_pages_per_seq=s["maxp"], w_uv=s["w_uv"])
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(spec, budget_s=12.0):
+    """Time the oracle on a bounded sample: repeated single-sequence steps until ~budget_s."""
+    s = oracle_sample(spec)
+    cols = (spec["L"] // spec["g"] + spec["R"]) if spec["mode"] == "shard" else (spec["L"] + spec["R"])
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_step(spec, s)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    bytes_done = n * s["T"] * cols * 2
+    return {"value": bytes_done / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": "%d oracle step(s) of 1 sequence x %d tokens (%s, all %d heads) in %.1f s; float64 numpy"
+                      % (n, s["T"], "shard 0" if spec["mode"] == "shard" else "all shards", spec["H"], dt)}
+
+
+def run_reference(args, spec, rank):
+    if rank != 0:
+        return None
+    s = oracle_sample(spec)
+    cols = (spec["L"] // spec["g"] + spec["R"]) if spec["mode"] == "shard" else (spec["L"] + spec["R"])
+    for _ in range(args.warmup):
+        oracle_step(spec, s)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(spec, s)
+    dt = (time.perf_counter() - t0) / args.steps
+    gbs = s["T"] * cols * 2 / dt / 1e9
+    sample = "each step: oracle append + decode of 1 sequence x %d tokens (of the %d-sequence workload)" % (
+        s["T"], spec["B"])
+    return {"metric": METRIC, "value": gbs, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(spec),
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def config_of(spec):
+    T = spec["T"]
+    return {"workload": spec["name"], "entry": "tpla_decode_shard(shard 0)" if spec["mode"] == "shard"
+            else ("mla_decode" if spec["g"] == 1 else "tpla_decode (all shards, on-chip sum)"),
+            "batch": spec["B"], "heads": spec["H"], "kv_lora_rank": spec["L"], "rope_dim": spec["R"],
+            "v_head_dim": spec["dv"], "shards_g": spec["g"],
+            "context": T if not isinstance(T, tuple) else "uniform[%d,%d]" % T,
+            "transform": {0: "none", 1: "hadamard", 2: "dense orthogonal (seeded QR)"}[spec["transform"]],
+            "page_size": 64, "step": "append 1 token/seq + split-KV attention + combine",
+            "l2": "inputs larger than L2 (no flush)"}
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="tpla_g2_dsv3_b16_32k")
+    ap.add_argument("--mode", default=None, choices=[None, "shard", "full"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    spec = workload_spec(args.workload)
+    if args.mode:
+        spec["mode"] = args.mode
+
+    rank, world, local = dist_init()
+    if args.impl == "reference":
+        line = run_reference(args, spec, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    r = run_gpu_arm(args, spec, rank, world, local)
+    if rank != 0:
+        return
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    value = r["total_cache"] / (r["ms"] * 1e-3) / 1e9
+    achieved = r["attn_bytes"] / (r["attn_ms"] * 1e-3) / 1e9
+    kernel_name = {1: "attn_simt", 2: "attn_sm100"}.get(r["kernel"], "unknown")
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms"], "us_per_step": r["ms"] * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_of(spec),
+        "hbm_frac_step": value / world / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(kernel_name, spec["name"]),
+                     "kernel": kernel_name + " (tpla_attention)", "peak_kind": peak_kind,
+                     "bytes_per_launch": r["attn_bytes"], "us_per_launch": r["attn_ms"] * 1e3},
+        "e2e": {"value": r["total_cache"] / (r["e2e_ms"] * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"]},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(spec)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
+    try:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+    except Exception:
+        pass

@@ -1,0 +1,324 @@
+// Host side of the C ABI declared in include/tpla.h: argument validation,
+// the split-KV plan, workspace carving, kernel dispatch and the device
+// status word.  Every check that can be made without the GPU runs before any
+// CUDA call, so a bad argument returns its status with nothing enqueued.
+#include "tpla_internal.cuh"
+
+#include <cmath>
+#include <cstdio>
+#include <mutex>
+
+namespace tpla {
+
+// Per-device status word (bits kStatusIndex, kStatusTimeout), set by kernels.
+__device__ unsigned int g_device_status;
+
+namespace {
+
+int g_opt_kernel = 0;        // TPLA_OPT_ATTENTION_KERNEL
+int g_opt_max_workers = 0;   // TPLA_OPT_MAX_WORKERS
+int g_opt_wait_limit = 0;    // TPLA_OPT_WAIT_LIMIT
+int g_opt_debug_stall = 0;   // TPLA_OPT_DEBUG_STALL
+int g_last_kernel = 0;       // TPLA_OPT_LAST_ATTENTION_KERNEL
+
+constexpr int kMinUnitsPerWorker = 6;   // keeps partial traffic small at batch 1
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mutex;
+unsigned* g_status_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int check_dims(const tpla_dims_t* d) {
+    if (!d) return TPLA_ERR_INVALID_ARG;
+    if (d->B < 0 || d->H <= 0 || d->L <= 0 || d->R <= 0 || d->dv <= 0 || d->g <= 0 ||
+        d->max_pages_per_seq <= 0 || d->num_pages <= 0)
+        return TPLA_ERR_INVALID_ARG;
+    if (!std::isfinite(d->softmax_scale)) return TPLA_ERR_INVALID_ARG;
+    if (d->page_size != kPage) return TPLA_ERR_UNSUPPORTED;
+    if (d->H > 128) return TPLA_ERR_UNSUPPORTED;
+    if (!(d->g == 1 || d->g == 2 || d->g == 4 || d->g == 8)) return TPLA_ERR_UNSUPPORTED;
+    if (!pow2(d->L) || d->L < 64 || d->L > 1024) return TPLA_ERR_UNSUPPORTED;
+    if (d->L % d->g) return TPLA_ERR_UNSUPPORTED;
+    const int Ls = d->L / d->g;
+    if (Ls < 32 || Ls > 512) return TPLA_ERR_UNSUPPORTED;
+    if (!(d->R == 16 || d->R == 32 || d->R == 64)) return TPLA_ERR_UNSUPPORTED;
+    if (d->dv % 8 || d->dv > 256) return TPLA_ERR_UNSUPPORTED;
+    if ((long long)d->max_pages_per_seq * kPage > (1ll << 30)) return TPLA_ERR_UNSUPPORTED;
+    return TPLA_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t ws_lse_bytes(const tpla_dims_t* d) {
+    return align_up((size_t)(kMaxWorkers + (size_t)d->B * d->g) * d->H * sizeof(float), 256);
+}
+
+size_t ws_bytes_for(const tpla_dims_t* d) {
+    const size_t slots = (size_t)kMaxWorkers + (size_t)d->B * d->g;
+    return 256 + ws_lse_bytes(d) + slots * d->H * (size_t)(d->L / d->g) * sizeof(float);
+}
+
+int device_info(unsigned** status, int* sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TPLA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return TPLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_status_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) return TPLA_ERR_CUDA;
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return TPLA_ERR_CUDA;
+        g_sm_count[dev] = n;
+        g_status_ptr[dev] = static_cast<unsigned*>(ptr);
+    }
+    if (status) *status = g_status_ptr[dev];
+    if (sms) *sms = g_sm_count[dev];
+    return TPLA_OK;
+}
+
+// Validation common to the decode stages.  shard == -1: all shards.
+int check_decode(const tpla_dims_t* d, int shard, const void* q, const void* q_pe, const void* ckv,
+                 const void* kpe, const int32_t* block_table, const int32_t* seq_lens,
+                 void* workspace, size_t ws_bytes) {
+    int st = check_dims(d);
+    if (st) return st;
+    if (shard < -1 || shard >= d->g) return TPLA_ERR_INVALID_ARG;
+    if (d->B == 0) return TPLA_OK;
+    if (!q || !q_pe || !ckv || !kpe || !seq_lens) return TPLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(q_pe) || !aligned16(ckv) || !aligned16(kpe) || !aligned16(seq_lens))
+        return TPLA_ERR_INVALID_ARG;
+    if (block_table && !aligned16(block_table)) return TPLA_ERR_INVALID_ARG;
+    if (!block_table && (long long)d->B * d->max_pages_per_seq > d->num_pages) return TPLA_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return TPLA_ERR_WORKSPACE;
+    if (ws_bytes < ws_bytes_for(d)) return TPLA_ERR_WORKSPACE;
+    return TPLA_OK;
+}
+
+int make_plan(const tpla_dims_t* d, int shard, Plan* p) {
+    unsigned* status = nullptr;
+    int sms = 0;
+    int st = device_info(&status, &sms);
+    if (st) return st;
+    p->B = d->B; p->H = d->H; p->L = d->L; p->R = d->R; p->dv = d->dv; p->g = d->g;
+    p->Ls = d->L / d->g;
+    p->gc = shard < 0 ? d->g : 1;
+    p->shard0 = shard < 0 ? 0 : shard;
+    p->max_pages = d->max_pages_per_seq;
+    p->num_pages = d->num_pages;
+    p->scale_log2 = d->softmax_scale * kLog2e;
+    p->status = status;
+    int cap = sms < kMaxWorkers ? sms : kMaxWorkers;
+    if (g_opt_max_workers > 0 && g_opt_max_workers < cap) cap = g_opt_max_workers;
+    const long long umax = (long long)p->gc * d->B * d->max_pages_per_seq;
+    long long w = (umax + kMinUnitsPerWorker - 1) / kMinUnitsPerWorker;
+    p->W = (int)(w < 1 ? 1 : (w > cap ? cap : w));
+    return TPLA_OK;
+}
+
+Workspace carve(void* workspace, const tpla_dims_t* d) {
+    char* base = static_cast<char*>(workspace) + 256;
+    Workspace w;
+    w.part_lse = reinterpret_cast<float*>(base);
+    w.part_o = reinterpret_cast<float*>(base + ws_lse_bytes(d));
+    return w;
+}
+
+int run_attention(const tpla_dims_t* d, int shard, const tpla_bf16* q, const tpla_bf16* q_pe,
+                  const tpla_bf16* ckv, const tpla_bf16* kpe, const int32_t* block_table,
+                  const int32_t* seq_lens, void* workspace, size_t ws_bytes, void* stream) {
+    int st = check_decode(d, shard, q, q_pe, ckv, kpe, block_table, seq_lens, workspace, ws_bytes);
+    if (st || d->B == 0) return st;
+    Plan p;
+    if ((st = make_plan(d, shard, &p))) return st;
+    Workspace w = carve(workspace, d);
+    auto bq = reinterpret_cast<const __nv_bfloat16*>(q);
+    auto bqp = reinterpret_cast<const __nv_bfloat16*>(q_pe);
+    auto bc = reinterpret_cast<const __nv_bfloat16*>(ckv);
+    auto bk = reinterpret_cast<const __nv_bfloat16*>(kpe);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    const bool tc_ok = sm100_supports(p);
+    if (g_opt_kernel == 2 && !tc_ok) return TPLA_ERR_UNSUPPORTED;
+    if (g_opt_kernel != 1 && tc_ok) {
+        e = launch_attention_sm100(p, bq, bqp, bc, bk, block_table, seq_lens, w, g_opt_wait_limit,
+                                   g_opt_debug_stall, s);
+        g_last_kernel = 2;
+    } else {
+        e = launch_attention_simt(p, bq, bqp, bc, bk, block_table, seq_lens, w, s);
+        g_last_kernel = 1;
+    }
+    if (e == cudaErrorNotSupported) return TPLA_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? TPLA_OK : TPLA_ERR_CUDA;
+}
+
+int run_combine(const tpla_dims_t* d, int shard, const int32_t* seq_lens, const tpla_bf16* w_uv,
+                float* out, void* workspace, size_t ws_bytes, void* stream) {
+    int st = check_dims(d);
+    if (st) return st;
+    if (shard < -1 || shard >= d->g) return TPLA_ERR_INVALID_ARG;
+    if (d->B == 0) return TPLA_OK;
+    if (!seq_lens || !out) return TPLA_ERR_INVALID_ARG;
+    if (w_uv && !aligned16(w_uv)) return TPLA_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return TPLA_ERR_WORKSPACE;
+    if (ws_bytes < ws_bytes_for(d)) return TPLA_ERR_WORKSPACE;
+    Plan p;
+    if ((st = make_plan(d, shard, &p))) return st;
+    cudaError_t e = launch_combine(p, seq_lens, reinterpret_cast<const __nv_bfloat16*>(w_uv), out,
+                                   carve(workspace, d), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TPLA_OK : TPLA_ERR_CUDA;
+}
+
+int run_decode(const tpla_dims_t* d, int shard, const tpla_bf16* q, const tpla_bf16* q_pe,
+               const tpla_bf16* ckv, const tpla_bf16* kpe, const int32_t* block_table,
+               const int32_t* seq_lens, const tpla_bf16* w_uv, float* out, void* workspace,
+               size_t ws_bytes, void* stream) {
+    int st = check_decode(d, shard, q, q_pe, ckv, kpe, block_table, seq_lens, workspace, ws_bytes);
+    if (st) return st;
+    if (d->B > 0 && !out) return TPLA_ERR_INVALID_ARG;
+    if (w_uv && !aligned16(w_uv)) return TPLA_ERR_INVALID_ARG;
+    if ((st = run_attention(d, shard, q, q_pe, ckv, kpe, block_table, seq_lens, workspace, ws_bytes, stream)))
+        return st;
+    return run_combine(d, shard, seq_lens, w_uv, out, workspace, ws_bytes, stream);
+}
+
+}  // namespace
+}  // namespace tpla
+
+using namespace tpla;
+
+extern "C" {
+
+const char* tpla_status_string(int status) {
+    switch (status) {
+        case TPLA_OK: return "TPLA_OK";
+        case TPLA_ERR_INVALID_ARG: return "TPLA_ERR_INVALID_ARG: null, negative or misaligned argument";
+        case TPLA_ERR_UNSUPPORTED: return "TPLA_ERR_UNSUPPORTED: size outside the supported set";
+        case TPLA_ERR_LAYOUT: return "TPLA_ERR_LAYOUT: cache layout does not match the call";
+        case TPLA_ERR_WORKSPACE: return "TPLA_ERR_WORKSPACE: workspace missing or too small";
+        case TPLA_ERR_CUDA: return "TPLA_ERR_CUDA: CUDA runtime error";
+        case TPLA_ERR_TIMEOUT: return "TPLA_ERR_TIMEOUT: a bounded device wait ran out";
+        case TPLA_ERR_INDEX: return "TPLA_ERR_INDEX: device-side index out of range";
+    }
+    return "unknown tpla status";
+}
+
+size_t tpla_decode_workspace_size(const tpla_dims_t* dims) {
+    if (check_dims(dims)) return 0;
+    return ws_bytes_for(dims);
+}
+
+int tpla_decode(const tpla_dims_t* dims, const tpla_bf16* q, const tpla_bf16* q_pe,
+                const tpla_bf16* ckv, const tpla_bf16* kpe, const int32_t* block_table,
+                const int32_t* seq_lens, const tpla_bf16* w_uv, float* out, void* workspace,
+                size_t ws_bytes, void* stream) {
+    return run_decode(dims, -1, q, q_pe, ckv, kpe, block_table, seq_lens, w_uv, out, workspace, ws_bytes,
+                      stream);
+}
+
+int tpla_decode_shard(const tpla_dims_t* dims, int shard, const tpla_bf16* q, const tpla_bf16* q_pe,
+                      const tpla_bf16* ckv, const tpla_bf16* kpe, const int32_t* block_table,
+                      const int32_t* seq_lens, const tpla_bf16* w_uv, float* out, void* workspace,
+                      size_t ws_bytes, void* stream) {
+    if (dims && (shard < 0 || shard >= dims->g)) return TPLA_ERR_INVALID_ARG;
+    return run_decode(dims, shard, q, q_pe, ckv, kpe, block_table, seq_lens, w_uv, out, workspace,
+                      ws_bytes, stream);
+}
+
+int mla_decode(const tpla_dims_t* dims, const tpla_bf16* q, const tpla_bf16* q_pe,
+               const tpla_bf16* ckv, const tpla_bf16* kpe, const int32_t* block_table,
+               const int32_t* seq_lens, const tpla_bf16* w_uv, float* out, void* workspace,
+               size_t ws_bytes, void* stream) {
+    if (!dims) return TPLA_ERR_INVALID_ARG;
+    if (dims->g != 1) return TPLA_ERR_LAYOUT;
+    return run_decode(dims, -1, q, q_pe, ckv, kpe, block_table, seq_lens, w_uv, out, workspace, ws_bytes,
+                      stream);
+}
+
+int tpla_attention(const tpla_dims_t* dims, int shard, const tpla_bf16* q, const tpla_bf16* q_pe,
+                   const tpla_bf16* ckv, const tpla_bf16* kpe, const int32_t* block_table,
+                   const int32_t* seq_lens, void* workspace, size_t ws_bytes, void* stream) {
+    return run_attention(dims, shard, q, q_pe, ckv, kpe, block_table, seq_lens, workspace, ws_bytes, stream);
+}
+
+int tpla_combine(const tpla_dims_t* dims, int shard, const int32_t* seq_lens, const tpla_bf16* w_uv,
+                 float* out, void* workspace, size_t ws_bytes, void* stream) {
+    return run_combine(dims, shard, seq_lens, w_uv, out, workspace, ws_bytes, stream);
+}
+
+int tpla_append_kv(const tpla_dims_t* dims, const tpla_bf16* latent_raw, const tpla_bf16* kpe_new,
+                   int transform, const float* R_dense, const float* norm_weight, float eps,
+                   const int32_t* positions, const int32_t* block_table, tpla_bf16* ckv_cache,
+                   tpla_bf16* kpe_cache, void* stream) {
+    int st = check_dims(dims);
+    if (st) return st;
+    if (transform < TPLA_TRANSFORM_NONE || transform > TPLA_TRANSFORM_DENSE) return TPLA_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return TPLA_ERR_INVALID_ARG;
+    if (dims->B == 0) return TPLA_OK;
+    if (!latent_raw || !kpe_new || !positions || !ckv_cache || !kpe_cache) return TPLA_ERR_INVALID_ARG;
+    if (transform == TPLA_TRANSFORM_DENSE && !R_dense) return TPLA_ERR_INVALID_ARG;
+    if (!aligned16(ckv_cache) || !aligned16(kpe_cache) || !aligned16(latent_raw) || !aligned16(kpe_new))
+        return TPLA_ERR_INVALID_ARG;
+    if (!block_table && (long long)dims->B * dims->max_pages_per_seq > dims->num_pages)
+        return TPLA_ERR_INVALID_ARG;
+    unsigned* status = nullptr;
+    if ((st = device_info(&status, nullptr))) return st;
+    cudaError_t e = launch_append(*dims, reinterpret_cast<const __nv_bfloat16*>(latent_raw),
+                                  reinterpret_cast<const __nv_bfloat16*>(kpe_new), transform, R_dense,
+                                  norm_weight, eps, positions, block_table,
+                                  reinterpret_cast<__nv_bfloat16*>(ckv_cache),
+                                  reinterpret_cast<__nv_bfloat16*>(kpe_cache), status,
+                                  static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return TPLA_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? TPLA_OK : TPLA_ERR_CUDA;
+}
+
+int tpla_check_device_status(void* stream) {
+    unsigned* status = nullptr;
+    int st = device_info(&status, nullptr);
+    if (st) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TPLA_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return TPLA_ERR_CUDA;
+    const unsigned zero = 0;
+    if (cudaMemcpy(status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return TPLA_ERR_CUDA;
+    if (v & kStatusTimeout) return TPLA_ERR_TIMEOUT;
+    if (v & kStatusIndex) return TPLA_ERR_INDEX;
+    return TPLA_OK;
+}
+
+int tpla_set_option(int option, int value) {
+    switch (option) {
+        case TPLA_OPT_ATTENTION_KERNEL:
+            if (value < 0 || value > 2) return TPLA_ERR_INVALID_ARG;
+            g_opt_kernel = value; return TPLA_OK;
+        case TPLA_OPT_MAX_WORKERS:
+            if (value < 0) return TPLA_ERR_INVALID_ARG;
+            g_opt_max_workers = value; return TPLA_OK;
+        case TPLA_OPT_WAIT_LIMIT:
+            if (value < 0) return TPLA_ERR_INVALID_ARG;
+            g_opt_wait_limit = value; return TPLA_OK;
+        case TPLA_OPT_DEBUG_STALL:
+            if (value < 0 || value > 1) return TPLA_ERR_INVALID_ARG;
+            g_opt_debug_stall = value; return TPLA_OK;
+    }
+    return TPLA_ERR_INVALID_ARG;
+}
+
+int tpla_get_option(int option) {
+    switch (option) {
+        case TPLA_OPT_ATTENTION_KERNEL: return g_opt_kernel;
+        case TPLA_OPT_MAX_WORKERS: return g_opt_max_workers;
+        case TPLA_OPT_WAIT_LIMIT: return g_opt_wait_limit;
+        case TPLA_OPT_DEBUG_STALL: return g_opt_debug_stall;
+        case TPLA_OPT_LAST_ATTENTION_KERNEL: return g_last_kernel;
+    }
+    return -1;
+}
+
+const char* tpla_version(void) { return "tpla-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

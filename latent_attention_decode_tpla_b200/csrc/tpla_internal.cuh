@@ -1,0 +1,184 @@
+// Internal declarations shared by the libtpla.so translation units.
+//
+// Split-KV schedule (not on the TPLA pages; it is how one GPU keeps all SMs
+// busy at small batch): the work of a call is a list of "units", one per
+// (sequence b, shard s of the call, 64-token tile), ordered b-major, then
+// shard, then tile.  Worker w (a CTA, or a CTA pair) takes the contiguous
+// unit range [lo(w), lo(w+1)) with lo(w) = floor(w * U / W).  Inside that
+// range each run of one (b, s) is a "segment"; it leaves one partial result
+// (normalised output rows + log2-sum-exp per head) in slot
+//     w                      if the segment starts the worker's range,
+//     W + b * gc + s         otherwise (the segment then starts at tile 0).
+// The combine kernel rebuilds the same lists from seq_lens alone, so the host
+// never needs the lengths and no kernel waits on another CTA.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/tpla.h"
+
+namespace tpla {
+
+constexpr int kPage = 64;            // tokens per cache page and per attention tile
+constexpr int kMaxWorkers = 160;     // workspace is sized for this many split-KV workers
+constexpr float kLog2e = 1.4426950408889634f;
+
+// device status bits (tpla_check_device_status)
+constexpr unsigned kStatusIndex = 1u;
+constexpr unsigned kStatusTimeout = 2u;
+
+struct Plan {
+    int B, H, L, R, dv, g;
+    int Ls;            // latent columns per shard (L / g)
+    int gc;            // shards handled by this call (g, or 1 for a single-shard call)
+    int shard0;        // first shard index of the call
+    int max_pages, num_pages;
+    int W;             // split-KV workers
+    float scale_log2;  // softmax_scale * log2(e)
+    unsigned* status;  // device status word (kStatus* bits)
+};
+
+struct Workspace {
+    float* part_lse;   // [slots][H]
+    float* part_o;     // [slots][H][Ls]
+};
+
+__host__ __device__ inline int num_slots(const Plan& p) { return p.W + p.B * p.gc; }
+
+__host__ __device__ inline long long unit_lo(long long w, long long U, long long W) {
+    return (w * U) / W;
+}
+
+// Worker that owns unit u (0 <= u < U): the largest w with lo(w) <= u.
+__host__ __device__ inline int unit_worker(long long u, long long U, long long W) {
+    return (int)(((u + 1) * W - 1) / U);
+}
+
+// Tokens of sequence b that are read: seq_lens[b] clamped to [0, 64 * max_pages];
+// a clamp is a caller error and is recorded in the device status.
+__device__ inline int effective_len(const int32_t* seq_lens, int b, int max_pages, unsigned* status) {
+    int T = __ldg(seq_lens + b);
+    int cap = max_pages * kPage;
+    if (T < 0 || T > cap) {
+        atomicOr(status, kStatusIndex);
+        T = T < 0 ? 0 : cap;
+    }
+    return T;
+}
+
+__device__ inline int tiles_of_len(int T) { return (T + kPage - 1) / kPage; }
+
+// Physical page of logical page `lp` of sequence b; -1 (recorded) if outside the cache.
+__device__ inline int page_lookup(const int32_t* block_table, int b, int lp, int max_pages, int num_pages,
+                                  unsigned* status) {
+    int page = block_table ? __ldg(block_table + (size_t)b * max_pages + lp) : b * max_pages + lp;
+    if (page < 0 || page >= num_pages) {
+        atomicOr(status, kStatusIndex);
+        return -1;
+    }
+    return page;
+}
+
+// Sum over b of gc * tiles(b), by one full warp (all 32 lanes call it).
+__device__ inline long long warp_total_units(const int32_t* seq_lens, int B, int max_pages, int gc) {
+    const int lane = threadIdx.x & 31;
+    long long acc = 0;
+    for (int base = 0; base < B; base += 32) {
+        int b = base + lane;
+        int n = 0;
+        if (b < B) {
+            int T = __ldg(seq_lens + b);
+            T = T < 0 ? 0 : (T > max_pages * kPage ? max_pages * kPage : T);
+            n = tiles_of_len(T);
+        }
+        acc += n;
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    return acc * gc;
+}
+
+// Position of unit u in (b, s, tile) coordinates, found by one full warp.
+// Returns b = B if u >= U.
+struct UnitPos { int b, s, tile, ntiles, T; };
+
+__device__ inline UnitPos warp_locate_unit(const int32_t* seq_lens, int B, int max_pages, int gc, long long u) {
+    const int lane = threadIdx.x & 31;
+    long long before = 0;                       // units of sequences < base
+    for (int base = 0; base < B; base += 32) {
+        int b = base + lane;
+        int n = 0;
+        if (b < B) {
+            int T = __ldg(seq_lens + b);
+            T = T < 0 ? 0 : (T > max_pages * kPage ? max_pages * kPage : T);
+            n = tiles_of_len(T) * gc;
+        }
+        long long incl = n;                     // inclusive scan over the 32 lanes
+        for (int o = 1; o < 32; o <<= 1) {
+            long long v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        long long chunk = __shfl_sync(0xffffffffu, incl, 31);
+        if (u < before + chunk) {
+            unsigned hit = __ballot_sync(0xffffffffu, b < B && u < before + incl);
+            int src = __ffs(hit) - 1;
+            long long excl = __shfl_sync(0xffffffffu, incl - n, src);
+            int nb = __shfl_sync(0xffffffffu, n, src);
+            UnitPos r;
+            r.b = base + src;
+            long long off = u - before - excl;
+            int per = nb / gc;
+            r.s = (int)(off / per);
+            r.tile = (int)(off % per);
+            r.ntiles = per;
+            int T = __ldg(seq_lens + r.b);
+            r.T = T < 0 ? 0 : (T > max_pages * kPage ? max_pages * kPage : T);
+            return r;
+        }
+        before += chunk;
+    }
+    UnitPos r; r.b = B; r.s = 0; r.tile = 0; r.ntiles = 0; r.T = 0;
+    return r;
+}
+
+// Advance a unit position by one unit (scalar; skips empty sequences).
+__device__ inline void advance_unit(UnitPos& p, const int32_t* seq_lens, int B, int max_pages, int gc) {
+    if (++p.tile < p.ntiles) return;
+    p.tile = 0;
+    if (++p.s < gc) return;
+    p.s = 0;
+    for (;;) {
+        if (++p.b >= B) { p.ntiles = 0; return; }
+        int T = __ldg(seq_lens + p.b);
+        T = T < 0 ? 0 : (T > max_pages * kPage ? max_pages * kPage : T);
+        p.T = T;
+        p.ntiles = tiles_of_len(T);
+        if (p.ntiles > 0) return;
+    }
+}
+
+// ---------------------------------------------------------------- launchers (one per .cu file)
+
+cudaError_t launch_attention_simt(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16* q_pe,
+                                  const __nv_bfloat16* ckv, const __nv_bfloat16* kpe,
+                                  const int32_t* block_table, const int32_t* seq_lens,
+                                  Workspace ws, cudaStream_t stream);
+
+// Returns cudaErrorNotSupported when the shape has no tcgen05 variant.
+cudaError_t launch_attention_sm100(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16* q_pe,
+                                   const __nv_bfloat16* ckv, const __nv_bfloat16* kpe,
+                                   const int32_t* block_table, const int32_t* seq_lens,
+                                   Workspace ws, int wait_limit, int debug_stall, cudaStream_t stream);
+bool sm100_supports(const Plan& p);
+
+cudaError_t launch_combine(const Plan& p, const int32_t* seq_lens, const __nv_bfloat16* w_uv,
+                           float* out, Workspace ws, cudaStream_t stream);
+
+cudaError_t launch_append(const tpla_dims_t& d, const __nv_bfloat16* latent_raw,
+                          const __nv_bfloat16* kpe_new, int transform, const float* R_dense,
+                          const float* norm_weight, float eps, const int32_t* positions,
+                          const int32_t* block_table, __nv_bfloat16* ckv, __nv_bfloat16* kpe,
+                          unsigned* status, cudaStream_t stream);
+
+}  // namespace tpla

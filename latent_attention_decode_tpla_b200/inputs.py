@@ -33,12 +33,32 @@ def _gen(seed, sub):
     return g
 
 
-def randn(shape, seed, sub, std=1.0, dtype=torch.bfloat16):
-    """N(0, std^2) samples drawn in float32 on the CPU, then cast (RN-even) to ``dtype``."""
-    x = torch.randn(*shape, generator=_gen(seed, sub), dtype=torch.float32)
-    if std != 1.0:
-        x = x * std
-    return x.to(dtype)
+def randn(shape, seed, sub, std=1.0, dtype=torch.bfloat16, chunk_elems=1 << 26):
+    """N(0, std^2) samples drawn in float32 on the CPU, then cast (RN-even) to ``dtype``.
+
+    Large tensors are drawn in slices along dim 0 from one generator, so the
+    values do not depend on the slice size beyond the fixed ``chunk_elems``.
+    """
+    shape = tuple(int(s) for s in shape)
+    gen = _gen(seed, sub)
+    n = 1
+    for s in shape:
+        n *= s
+    if n <= chunk_elems or len(shape) == 1:
+        x = torch.randn(*shape, generator=gen, dtype=torch.float32)
+        if std != 1.0:
+            x = x * std
+        return x.to(dtype)
+    out = torch.empty(shape, dtype=dtype)
+    row = n // shape[0]
+    step = max(1, chunk_elems // row)
+    for i in range(0, shape[0], step):
+        j = min(shape[0], i + step)
+        x = torch.randn((j - i,) + shape[1:], generator=gen, dtype=torch.float32)
+        if std != 1.0:
+            x = x * std
+        out[i:j] = x.to(dtype)
+    return out
 
 
 def random_orthogonal(L, seed):

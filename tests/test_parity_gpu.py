@@ -1,0 +1,192 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Inputs are seeded and identical on both sides (bf16 values).  Tolerances on
+the fp32 outputs: max-abs <= 2e-2 and relative RMS <= 1e-3.  Small cases span
+several 64-token tiles, ragged tails and empty sequences; the benchmark
+configurations run at full size, with the oracle evaluated on a sample of
+sequences where the whole batch would take too long on the CPU.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import gpu_harness as hx
+from oracle import tpla_ref as ref
+from latent_attention_decode_tpla_b200 import inputs as gen
+from latent_attention_decode_tpla_b200 import tpla
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = ["simt", "sm100"]
+
+
+def _kernel_or_skip(d, kernel):
+    if kernel == "sm100" and not hx.sm100_available(d):
+        pytest.skip("no tcgen05 variant for this shape")
+
+
+def _case(B, H, L, R, dv, g, lens, seed, transform=None, **kw):
+    d = gen.make_workload(B=B, H=H, L=L, R=R, dv=dv, g=g, seq_lens=lens, seed=seed, extra_pages=5,
+                          cache_values="none" if transform is not None else "normal", **kw)
+    if transform is not None:
+        Rd = gen.random_orthogonal(L, seed) if transform == ref.TRANSFORM_DENSE else None
+        hx.oracle_fill_cache(d, transform, Rd)
+    return d
+
+
+# ------------------------------------------------------------------ tiny TPLA decode (H8 L64 R16 dv32, g=2, 128 tokens)
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_tiny_g2_hadamard(kernel):
+    spec = gen.WORKLOADS["tiny_g2"]
+    d = _case(spec["B"], spec["H"], spec["L"], spec["R"], spec["dv"], spec["g"], [spec["T"]], 0,
+              transform=ref.TRANSFORM_HADAMARD, **spec["stds"])
+    _kernel_or_skip(d, kernel)
+    scale = gen.softmax_scale(spec)
+    hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "tiny out")
+    hx.assert_close(hx.run_gpu(d, scale, with_wuv=False, kernel=kernel),
+                    hx.run_oracle(d, scale, with_wuv=False), "tiny latent")
+    tot = 0
+    for s in range(2):
+        got = hx.run_gpu(d, scale, mode="shard", shard=s, kernel=kernel)
+        hx.assert_close(got, hx.run_oracle(d, scale, mode="shard", shard=s), "tiny shard %d" % s)
+        tot = tot + got
+        hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=s, with_wuv=False, kernel=kernel),
+                        hx.run_oracle(d, scale, mode="shard", shard=s, with_wuv=False), "tiny shard latent")
+    # the sum of the per-rank terms is the full result (fp32 reassociation only)
+    np.testing.assert_allclose(tot, hx.run_gpu(d, scale, kernel=kernel), rtol=0, atol=1e-5)
+
+
+# ------------------------------------------------------------------ ragged small cases
+
+RAGGED = [0, 1, 63, 64, 65, 200, 7, 129]
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("H,L,R,dv,g", [
+    (8, 64, 16, 32, 2), (128, 512, 64, 128, 1), (128, 512, 64, 128, 2), (64, 512, 64, 128, 4),
+    (100, 512, 64, 128, 2), (128, 512, 64, 128, 8), (16, 256, 32, 64, 2), (64, 128, 16, 32, 4),
+])
+def test_ragged_batch(kernel, H, L, R, dv, g):
+    d = _case(len(RAGGED), H, L, R, dv, g, RAGGED, seed=3 + H + g)
+    _kernel_or_skip(d, kernel)
+    scale = 1 / math.sqrt(128 + R)
+    want = hx.run_oracle(d, scale)
+    hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), want, "out")
+    assert np.all(hx.run_gpu(d, scale, kernel=kernel)[0] == 0.0)          # empty sequence
+    hx.assert_close(hx.run_gpu(d, scale, with_wuv=False, kernel=kernel), hx.run_oracle(d, scale, with_wuv=False),
+                    "latent")
+    s = g - 1
+    hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=s, kernel=kernel),
+                    hx.run_oracle(d, scale, mode="shard", shard=s), "shard")
+    # identity page layout (block_table = NULL) on an unshuffled cache
+    d2 = gen.make_workload(B=3, H=H, L=L, R=R, dv=dv, g=g, seq_lens=[70, 0, 130], seed=9, shuffle=False)
+    hx.assert_close(hx.run_gpu(d2, scale, block_table=False, kernel=kernel), hx.run_oracle(d2, scale),
+                    "identity layout")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("workers", [1, 2, 3, 7, 0])
+def test_split_schedule_invariance(kernel, workers):
+    """Any number of split-KV workers gives the same result (segments cross workers and sequences)."""
+    d = _case(5, 128, 512, 64, 128, 2, [300, 1, 0, 640, 65], seed=17)
+    _kernel_or_skip(d, kernel)
+    scale = 1 / math.sqrt(192)
+    old = tpla.get_option(tpla.OPT_MAX_WORKERS)
+    tpla.set_option(tpla.OPT_MAX_WORKERS, workers)
+    try:
+        got = hx.run_gpu(d, scale, kernel=kernel)
+        got_s = hx.run_gpu(d, scale, mode="shard", shard=1, kernel=kernel)
+    finally:
+        tpla.set_option(tpla.OPT_MAX_WORKERS, old)
+    hx.assert_close(got, hx.run_oracle(d, scale), "workers=%d" % workers)
+    hx.assert_close(got_s, hx.run_oracle(d, scale, mode="shard", shard=1), "shard workers=%d" % workers)
+
+
+# ------------------------------------------------------------------ benchmark configurations, full size
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_mla_g1_dsv3_4k(kernel):
+    spec = gen.WORKLOADS["mla_g1_dsv3_b1_4k"]
+    d = _case(1, 128, 512, 64, 128, 1, [4096], 1, transform=ref.TRANSFORM_HADAMARD)
+    _kernel_or_skip(d, kernel)
+    scale = gen.softmax_scale(spec)
+    want = hx.run_oracle(d, scale)
+    hx.assert_close(hx.run_gpu(d, scale, mode="mla", kernel=kernel), want, "mla_decode")
+    hx.assert_close(hx.run_gpu(d, scale, mode="full", kernel=kernel), want, "tpla_decode g=1")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_tpla_g2_dsv3_b1_32k(kernel):
+    spec = gen.WORKLOADS["tpla_g2_dsv3_b1_32k"]
+    d = _case(1, 128, 512, 64, 128, 2, [32768], 2)
+    _kernel_or_skip(d, kernel)
+    scale = gen.softmax_scale(spec)
+    hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=0, kernel=kernel),
+                    hx.run_oracle(d, scale, mode="shard", shard=0), "shard 0")
+    hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "all shards")
+
+
+def _sampled(d, scale, batch, kernel, modes=("shard", "full")):
+    for mode in modes:
+        got = hx.run_gpu(d, scale, mode=mode, shard=0, kernel=kernel)
+        want = hx.run_oracle(d, scale, mode=mode, shard=0, batch=batch)
+        hx.assert_close(got[batch], want, "%s sampled %s" % (mode, batch))
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_tpla_g2_dsv3_b16_32k(kernel):
+    spec = gen.WORKLOADS["tpla_g2_dsv3_b16_32k"]
+    d = _case(16, 128, 512, 64, 128, 2, [32768] * 16, 3)
+    _kernel_or_skip(d, kernel)
+    _sampled(d, gen.softmax_scale(spec), [0, 9, 15], kernel)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_tpla_g4_kimi_b8_32k(kernel):
+    spec = gen.WORKLOADS["tpla_g4_kimi_b8_32k"]
+    d = _case(8, 64, 512, 64, 128, 4, [32768] * 8, 4)
+    _kernel_or_skip(d, kernel)
+    _sampled(d, gen.softmax_scale(spec), [0, 5], kernel)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_mixed_b64_paged_with_append(kernel):
+    """DeepSeek-V3 shape, g=2: 64 sequences of 1K..64K tokens on a shuffled page table, plus one appended token each."""
+    spec = gen.WORKLOADS["tpla_g2_dsv3_b64_mixed"]
+    lens = gen.workload_seq_lens(spec, seed=0)
+    d = gen.make_workload(B=64, H=128, L=512, R=64, dv=128, g=2, seq_lens=lens, seed=5)
+    _kernel_or_skip(d, kernel)
+    scale = gen.softmax_scale(spec)
+    dev = hx.to_device(d)
+    dims = hx.dims_of(d, scale)
+    tpla.append_kv(dims, dev["x_new"], dev["kpe_new"], tpla.TRANSFORM_HADAMARD, None, None, 1e-6,
+                   dev["seq_lens"], dev["block_table"], dev["ckv"], dev["kpe"])
+    torch.cuda.synchronize()
+    assert tpla.check_device_status() == tpla.TPLA_OK
+    # the oracle appends the same tokens into its own copy of the cache
+    batch = [int(lens.argmax()), int(lens.argmin()), 17]
+    ckv = hx.to64(d["ckv"])
+    kpe = hx.to64(d["kpe"])
+    bt = d["block_table"].numpy()
+    ref.append_kv(hx.to64(d["x_new"]), hx.to64(d["kpe_new"]), lens.numpy(), bt, ckv, kpe, g=2,
+                  max_pages_per_seq=d["max_pages_per_seq"], transform=ref.TRANSFORM_HADAMARD, eps=1e-6)
+    d_or = dict(d)
+    d_or["ckv"] = torch.from_numpy(ckv).to(torch.bfloat16)
+    d_or["kpe"] = torch.from_numpy(kpe).to(torch.bfloat16)
+    d_or["seq_lens"] = lens + 1
+    dev["seq_lens"] = (lens + 1).cuda()
+    # appended rows agree with the oracle's within one bf16 ulp
+    for b in batch:
+        page, slot = bt[b, int(lens[b]) // 64], int(lens[b]) % 64
+        g_row = dev["ckv"][page, :, slot].cpu().to(torch.float64).numpy()
+        o_row = ckv[page, :, slot]
+        assert np.all(np.abs(g_row - o_row) <= np.abs(o_row) * 2.0 ** -7 + 1e-30)
+    # end to end: GPU append + GPU decode against oracle append + oracle decode
+    for mode in ("full", "shard"):
+        got = hx.run_gpu(d_or, scale, mode=mode, shard=0, dev=dev, kernel=kernel)
+        want = hx.run_oracle(d_or, scale, mode=mode, shard=0, batch=batch)
+        hx.assert_close(got[batch], want, "mixed %s" % mode)
