@@ -74,10 +74,13 @@ def run_gpu(d, scale, mode="full", shard=0, with_wuv=True, dev=None, block_table
             tpla.mla_decode(dims, dev["q"], dev["q_pe"], dev["ckv"], dev["kpe"], bt, dev["seq_lens"], w, out, ws)
         else:
             raise ValueError(mode)
+        used = tpla.get_option(tpla.OPT_LAST_ATTENTION_KERNEL)
     finally:
         tpla.set_option(tpla.OPT_ATTENTION_KERNEL, old)
     torch.cuda.synchronize()
     assert tpla.check_device_status() == tpla.TPLA_OK
+    if kernel is not None:
+        assert used == KERNELS[kernel], "asked for %s, ran kernel %d" % (kernel, used)
     return to64(out)
 
 
