@@ -252,6 +252,7 @@ def gpu_step(w, spec, ev_attn=None):
 
 
 def run_gpu_arm(args, spec, rank, world, local):
+    """Times K steps (CUDA events on the launching stream), then K end-to-end steps."""
     import torch
     from latent_attention_decode_tpla_b200 import inputs as gen
     from latent_attention_decode_tpla_b200 import tpla
@@ -298,7 +299,7 @@ def run_gpu_arm(args, spec, rank, world, local):
     torch.cuda.synchronize()
     barrier()
     e_start.record(stream)
-    for _ in range(K):
+    for _ in range(0 if args.no_e2e else K):
         for k, t in host.items():
             w[k].copy_(t, non_blocking=True)
         gpu_step(w, spec)
@@ -308,7 +309,7 @@ def run_gpu_arm(args, spec, rank, world, local):
         _ = float(out_host[0, 0, 0])
     e_end.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / K)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / K) if not args.no_e2e else float("nan")
     st = tpla.check_device_status()
     if st != tpla.TPLA_OK:
         raise RuntimeError("device status after timing: " + tpla.status_string(st))
@@ -430,11 +431,16 @@ def main():
     ap.add_argument("--workload", default="tpla_g2_dsv3_b16_32k")
     ap.add_argument("--mode", default=None, choices=[None, "shard", "full"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     spec = workload_spec(args.workload)
     if args.mode:
         spec["mode"] = args.mode
+    if args.batch:
+        spec["B"] = args.batch
+        spec["name"] = spec["name"] + "_batch%d" % args.batch
 
     rank, world, local = dist_init()
     if args.impl == "reference":

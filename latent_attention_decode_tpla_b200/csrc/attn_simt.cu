@@ -166,7 +166,8 @@ cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16*
                      const int32_t* seq_lens, Workspace ws, cudaStream_t stream) {
     const size_t smem = sizeof(SimtSmem<LS, RD>);
     auto kern = attn_simt_kernel<LS, RD>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static unsigned long long attr_done = 0;
+    cudaError_t e = set_smem_once(kern, smem, &attr_done);
     if (e != cudaSuccess) return e;
     dim3 grid(p.W, (p.H + kHG - 1) / kHG);
     kern<<<grid, kThreads, smem, stream>>>(p, q, q_pe, ckv, kpe, bt, seq_lens, ws);

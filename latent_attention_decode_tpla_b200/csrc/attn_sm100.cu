@@ -16,33 +16,48 @@
 //     O[h, :] += P[h, t] . C_s[t, :]                M=128, N=Ls,  K=64
 // One 64-token tile is TMA-loaded once into 128B-swizzled shared memory and
 // is the K-major B operand of the first MMA and the MN-major B operand of
-// the second.  Q and P are the A operands and live in tensor memory, so the
-// shared-memory bandwidth goes to the cache stream only.  O (fp32) and S
-// (fp32) accumulate in tensor memory.
+// the second.
 //
-// Precision: QK^T multiplies the bf16 inputs as they are.  For PV the
-// probabilities are rounded to fp16 (11 significant bits) rather than bf16
-// (8 bits): rounding P to bf16 alone costs about 1.2e-3 relative RMS error on
-// outputs of short sequences, fp16 about 1.5e-4.  One MMA never mixes the
-// two types, so after QK^T of a tile has completed, the softmax warps convert
-// that tile's latent rows in shared memory from bf16 to fp16 in place (each
-// bf16 value of the RMS-normalised cache is exactly an fp16 value unless its
-// magnitude is below 2^-14), zero the rows past the end of the sequence, and
-// only then release the tile to PV.
+// Operand placement (tensor memory holds 512 columns of 128 lanes):
+//   tensor memory: O (Ls columns, fp32), two S buffers (64 columns each,
+//                  fp32), and the latent part of Q (Ls/2 columns, bf16
+//                  pairs) as the A operand of the first Ls/16 QK^T steps;
+//   shared memory: the RoPE part of Q (A operand of the last R/16 QK^T
+//                  steps) and two P buffers (A operand of PV), all in the
+//                  128B-swizzled K-major layout.
+// With two S and two P buffers the MMA warp issues QK^T(j+1) before PV(j):
+// the softmax of tile j has the time of PV(j-1) + QK^T(j+1) to produce P(j)
+// before the tensor pipe needs it.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads into a ring of NST
-// stages; warp 1 allocates tensor memory and issues the MMAs (one thread);
-// warps 2-5 own the 128 TMEM lanes (one head row per thread) and do the
-// softmax, the O rescale, the P store and the epilogue.  The MMA warp issues
-// QK^T of tile j before PV of tile j-1 so the tensor pipe works while the
-// softmax warps exponentiate.  O is rescaled only when a row's running
-// maximum grows by more than 8 (log2 units); a stale maximum only bounds
-// p by 2^8, which fp32 holds exactly enough.
+// Precision: QK^T multiplies the bf16 inputs as they are.  PV multiplies the
+// probabilities P, rounded to 16 bits, by the latent tile.  Rounding P to
+// bf16 (8 significant bits) gives outputs with about 1.2e-3 relative RMS
+// error on sequences of a few hundred tokens, falling to 3-7e-4 at 4K-32K
+// tokens (the output's systematic part grows with length while the rounding
+// noise averages out).  So a segment of a sequence shorter than
+// kExactPVBelow tokens runs PV in fp16 (11 bits, about 1.5e-4): one MMA never
+// mixes the two types, so after QK^T of such a tile has completed the softmax
+// warps convert its latent rows in shared memory from bf16 to fp16 in place
+// (each bf16 value of the RMS-normalised cache is exactly an fp16 value
+// unless its magnitude is below 2^-14).  Longer sequences keep the bf16 tile
+// and bf16 P, which costs no extra shared-memory traffic.  In both modes the
+// rows past the end of the sequence are zeroed before PV reads the tile.
 //
-// Every wait is bounded in time (globaltimer); a wait that runs out records
+// Warp roles (320 threads): warp 0 issues TMA loads into a ring of NST
+// stages (page-table entries fetched a few tiles ahead); warp 1 allocates
+// tensor memory and issues the MMAs (one thread); warps 2-9 are two softmax
+// warpgroups.  Both own all 128 TMEM lanes (one head row per thread);
+// warpgroup 0 takes score columns 0-31 of every tile, warpgroup 1 columns
+// 32-63, and they agree on each row's running maximum through a per-tile
+// exchange.  Each warpgroup rescales, and finally writes, its half of the O
+// columns.  O is rescaled only when a row's running maximum grows by more
+// than 8 (log2 units); a stale maximum only bounds p by 2^8.
+//
+// Every wait is bounded in time (SM clock cycles); a wait that runs out records
 // TPLA_ERR_TIMEOUT in the device status word, sets a CTA-wide abort flag so
 // all roles stop, and the kernel drains its TMA loads and MMAs before it
-// frees tensor memory and returns.
+// frees tensor memory and returns.  No role waits on a plain CTA barrier
+// while another may have stopped.
 #include "tpla_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -54,34 +69,45 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kSoftmaxWarp0 = 2;
+constexpr int kSoftmaxWarps = 8;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
+constexpr int kExactPVBelow = 8192;           // sequences shorter than this run PV in fp16
+constexpr int kPageAhead = 4;                 // page-table entries the producer loads ahead
 
 template <int LS, int RD, int NST>
 struct Cfg {
     static constexpr int kChunk = 64 * 128;                   // one 64-row x 128-byte swizzled chunk
     static constexpr int kChunksC = LS / 64;
-    static constexpr int kChunksK = RD / 64;
-    static constexpr int kStageBytes = (kChunksC + kChunksK) * kChunk;
-    static constexpr int kK = LS + RD;                         // QK^T contraction length
+    static constexpr int kStageBytes = (kChunksC + 1) * kChunk;   // latent chunks + the RoPE chunk
+    static constexpr int kPBytes = 128 * 128;                  // one P buffer: 128 rows x 64 tokens x 2 B
+    static constexpr int kQpeBytes = 128 * 128;                // RoPE query: 128 rows x 64 x 2 B
     static constexpr int kColO = 0;
-    static constexpr int kColS = LS;
-    static constexpr int kColP = LS + 64;
-    static constexpr int kColQ = LS + 96;
-    static constexpr int kColsUsed = kColQ + kK / 2;
+    static constexpr int kColS = LS;                           // two buffers of 64 columns
+    static constexpr int kColQ = LS + 128;                     // latent query, LS/2 columns
+    static constexpr int kColsUsed = kColQ + LS / 2;
     static constexpr int kTmemCols = kColsUsed <= 128 ? 128 : (kColsUsed <= 256 ? 256 : 512);
+    static constexpr int kStepsC = LS / 16;                    // QK^T steps over the latent
+    static constexpr int kStepsR = RD / 16;                    // QK^T steps over the RoPE key
     static constexpr uint32_t kIdescQK = idesc_f16kind(128, 64, false, true);    // bf16 x bf16
-    static constexpr uint32_t kIdescPV = idesc_f16kind(128, LS, true, false);    // fp16 x fp16
+    static constexpr uint32_t kIdescPVf16 = idesc_f16kind(128, LS, true, false);  // fp16 x fp16
+    static constexpr uint32_t kIdescPVbf16 = idesc_f16kind(128, LS, true, true);  // bf16 x bf16
+    static constexpr int kCvt = kChunksC * kPage * 8 / (kSoftmaxWarps * 32);      // 16-byte pieces per thread
+    static constexpr size_t kSmem = 1024 + (size_t)NST * kStageBytes + 2 * kPBytes + kQpeBytes;
     static_assert(kColsUsed <= 512, "tensor memory");
     static_assert(LS % 64 == 0 && RD == 64, "tile shape");
+    static_assert(kCvt >= 1 && kChunksC * kPage * 8 % (kSoftmaxWarps * 32) == 0, "conversion split");
 };
 
 template <int NST>
 struct Bars {
     uint64_t full[NST];
     uint64_t empty[NST];
-    uint64_t s_full, s_free, p_full, o_done, q_full, o_free, drain, never;
+    uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+    uint64_t q_full, o_free, xmax, xsum, drain, never;
+    float xmax_buf[2][2][128];     // [tile parity][warpgroup][row]
+    float xsum_buf[2][2][128];     // [segment parity][warpgroup][row]
     uint32_t tmem_base;
     volatile int abort;
 };
@@ -89,16 +115,17 @@ struct Bars {
 struct Waiter {
     volatile int* abort;
     unsigned* status;
-    uint64_t limit_ns;
+    uint64_t limit_cycles;
 
     // true when the phase of `parity` completed; false on abort or time-out
+    // (the limit is counted in SM clock cycles: reading %globaltimer in the loop is slow)
     __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
         if (mbar_try_wait(bar, parity)) return true;
-        const uint64_t t0 = globaltimer_ns();
+        const long long t0 = clock64();
         for (;;) {
             if (mbar_try_wait(bar, parity)) return true;
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > limit_ns) {
+            if ((uint64_t)(clock64() - t0) > limit_cycles) {
                 atomicOr(status, kStatusTimeout);
                 *abort = 1;
                 return false;
@@ -115,6 +142,17 @@ __device__ __forceinline__ SegFlags seg_flags(long long u, long long lo, long lo
     return {u == lo || pos.tile == 0, u == hi - 1 || pos.tile == pos.ntiles - 1};
 }
 
+// warp-collective: all lanes of the warp arrive through lane 0 after their prior writes
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// byte offset of 16-byte piece `c` of row `r` in a 128-row, 128B-swizzled K-major operand
+__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
 template <int LS, int RD, int NST>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_k, Plan p,
@@ -123,9 +161,15 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                   uint64_t wait_ns, int debug_stall) {
     using C = Cfg<LS, RD, NST>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    auto& bars = *reinterpret_cast<Bars<NST>*>(smem + NST * C::kStageBytes);
+    // 1024-byte aligned base, by pointer arithmetic on the shared array so that every access
+    // derived from it stays a shared-memory access
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint8_t* p_smem = smem + NST * C::kStageBytes;          // two P buffers
+    uint8_t* qpe_smem = p_smem + 2 * C::kPBytes;            // RoPE query
+    auto& bars = *reinterpret_cast<Bars<NST>*>(qpe_smem + C::kQpeBytes);
     const uint32_t stage0 = smem_addr(smem);
+    const uint32_t p_addr = smem_addr(p_smem);
+    const uint32_t qpe_addr = smem_addr(qpe_smem);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int w = blockIdx.x;
@@ -136,18 +180,23 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     const long long lo = unit_lo(w, U, p.W), hi = unit_lo(w + 1, U, p.W);
     if (lo >= hi) return;
     const UnitPos pos0 = warp_locate_unit(seq_lens, p.B, p.max_pages, p.gc, lo);
+    const long long n = hi - lo;                            // tiles of this worker
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) {
             mbar_init(smem_addr(&bars.full[i]), 1);
             mbar_init(smem_addr(&bars.empty[i]), 1);
         }
-        mbar_init(smem_addr(&bars.s_full), 1);
-        mbar_init(smem_addr(&bars.s_free), 4);
-        mbar_init(smem_addr(&bars.p_full), 4);
-        mbar_init(smem_addr(&bars.o_done), 1);
-        mbar_init(smem_addr(&bars.q_full), 4);
-        mbar_init(smem_addr(&bars.o_free), 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_addr(&bars.s_full[i]), 1);
+            mbar_init(smem_addr(&bars.s_free[i]), kSoftmaxWarps);
+            mbar_init(smem_addr(&bars.p_full[i]), kSoftmaxWarps);
+            mbar_init(smem_addr(&bars.o_done[i]), 1);
+        }
+        mbar_init(smem_addr(&bars.q_full), kSoftmaxWarps);
+        mbar_init(smem_addr(&bars.o_free), kSoftmaxWarps);
+        mbar_init(smem_addr(&bars.xmax), kSoftmaxWarps);
+        mbar_init(smem_addr(&bars.xsum), kSoftmaxWarps);
         mbar_init(smem_addr(&bars.drain), 1);
         mbar_init(smem_addr(&bars.never), 1);
         bars.abort = 0;
@@ -162,19 +211,34 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
-    const Waiter wt{&bars.abort, p.status, wait_ns};
+    // 2 cycles per nanosecond bounds the clock from above (B200 runs at most 1.965 GHz)
+    const Waiter wt{&bars.abort, p.status, wait_ns * 2};
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             UnitPos pos = pos0;
+            // page-table entries are loaded kPageAhead units ahead of their TMA issue
+            UnitPos ahead = pos0;
+            int pg[kPageAhead];
+#pragma unroll
+            for (int k = 0; k < kPageAhead; ++k) {
+                pg[k] = k < n ? page_lookup(block_table, ahead.b, ahead.tile, p.max_pages, p.num_pages, p.status) : -1;
+                if (k < n) advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
+            }
             long long j = 0;
-            for (long long u = lo; u < hi; ++u, ++j) {
+            for (; j < n; ++j) {
                 const int st = (int)(j % NST);
                 const uint32_t use = (uint32_t)(j / NST);
+                const int page = pg[0];
+#pragma unroll
+                for (int k = 0; k + 1 < kPageAhead; ++k) pg[k] = pg[k + 1];
+                if (j + kPageAhead < n) {
+                    pg[kPageAhead - 1] = page_lookup(block_table, ahead.b, ahead.tile, p.max_pages, p.num_pages, p.status);
+                    advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
+                }
                 if (use > 0 && !wt.wait(smem_addr(&bars.empty[st]), (use - 1) & 1)) break;
                 const int shard = p.shard0 + pos.s;
-                const int page = page_lookup(block_table, pos.b, pos.tile, p.max_pages, p.num_pages, p.status);
                 // an invalid page reads rows past the end of the tensor: TMA fills zeros
                 const int yc = page >= 0 ? (page * p.g + shard) * kPage : p.num_pages * p.g * kPage;
                 const int yk = page >= 0 ? page * kPage : p.num_pages * kPage;
@@ -187,8 +251,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 advance_unit(pos, seq_lens, p.B, p.max_pages, p.gc);
             }
             // drain: the last use of every stage must have landed before the CTA exits
-            const long long issued = j;
-            for (long long t = issued - NST < 0 ? 0 : issued - NST; t < issued; ++t) {
+            for (long long t = j - NST < 0 ? 0 : j - NST; t < j; ++t) {
                 const int st = (int)(t % NST);
                 // bounded wait that ignores the abort flag (the copy is in flight either way)
                 const uint64_t t0 = globaltimer_ns();
@@ -206,48 +269,73 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         if (lane == 0) {
             bool ok = true;
             if (debug_stall) ok = wt.wait(smem_addr(&bars.never), 0);   // nothing arrives: exercises the time-out
-            UnitPos pos = pos0;
-            long long j = 0;
-            int seg = -1;
-            bool prev_end = true, prev_first = false;
-            int prev_seg = -1;
-            auto issue_pv = [&](long long t, bool first, int tseg) -> bool {
-                if (!wt.wait(smem_addr(&bars.p_full), (uint32_t)(t & 1))) return false;
-                if (first && tseg > 0 && !wt.wait(smem_addr(&bars.o_free), (uint32_t)((tseg - 1) & 1))) return false;
-                tc_fence_after();
-                const uint32_t sb = stage0 + (int)(t % NST) * C::kStageBytes;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(sb + kk * 2048, C::kChunk, 1024);
-                    mma_ts(tmem + C::kColO, tmem + C::kColP + kk * 8, bd, C::kIdescPV, (first && kk == 0) ? 0u : 1u);
-                }
-                mma_commit(smem_addr(&bars.empty[(int)(t % NST)]));
-                mma_commit(smem_addr(&bars.o_done));
-                return true;
-            };
-            for (long long u = lo; ok && u < hi; ++u, ++j) {
-                const SegFlags f = seg_flags(u, lo, hi, pos);
+            // QK^T runs one tile ahead of PV, each with its own cursor over the worker's tiles
+            UnitPos qpos = pos0;
+            int qseg = -1;
+            auto issue_qk = [&](long long t) -> bool {
+                const SegFlags f = seg_flags(lo + t, lo, hi, qpos);
                 if (f.begin) {
-                    ++seg;
-                    if (!wt.wait(smem_addr(&bars.q_full), (uint32_t)(seg & 1))) break;
+                    ++qseg;
+                    if (!wt.wait(smem_addr(&bars.q_full), (uint32_t)(qseg & 1))) return false;
                 }
-                const int st = (int)(j % NST);
-                if (!wt.wait(smem_addr(&bars.full[st]), (uint32_t)((j / NST) & 1))) break;
-                if (j > 0 && !wt.wait(smem_addr(&bars.s_free), (uint32_t)((j - 1) & 1))) break;
+                const int st = (int)(t % NST);
+                if (!wt.wait(smem_addr(&bars.full[st]), (uint32_t)((t / NST) & 1))) return false;
+                const int b = (int)(t & 1);
+                if (t >= 2 && !wt.wait(smem_addr(&bars.s_free[b]), (uint32_t)(((t >> 1) - 1) & 1))) return false;
                 tc_fence_after();
                 const uint32_t sb = stage0 + st * C::kStageBytes;
+                const uint32_t d = tmem + C::kColS + b * 64;
 #pragma unroll
-                for (int kk = 0; kk < C::kK / 16; ++kk) {
+                for (int kk = 0; kk < C::kStepsC; ++kk) {
                     const uint64_t bd = smem_desc_sw128(sb + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024);
-                    mma_ts(tmem + C::kColS, tmem + C::kColQ + kk * 8, bd, C::kIdescQK, kk > 0 ? 1u : 0u);
+                    mma_ts(d, tmem + C::kColQ + kk * 8, bd, C::kIdescQK, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(smem_addr(&bars.s_full));
-                if (j > 0 && !prev_end && !issue_pv(j - 1, prev_first, prev_seg)) break;
-                if (f.end && !issue_pv(j, f.begin, seg)) break;
-                prev_end = f.end;
-                prev_first = f.begin;
-                prev_seg = seg;
-                advance_unit(pos, seq_lens, p.B, p.max_pages, p.gc);
+#pragma unroll
+                for (int kk = 0; kk < C::kStepsR; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(qpe_addr + kk * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(sb + C::kChunksC * C::kChunk + kk * 32, 16, 1024);
+                    mma_ss(d, ad, bd, C::kIdescQK, 1u);
+                }
+                mma_commit(smem_addr(&bars.s_full[b]));
+                advance_unit(qpos, seq_lens, p.B, p.max_pages, p.gc);
+                return true;
+            };
+            // PV cursor
+            UnitPos vpos = pos0;
+            int vseg = -1;
+            bool vexact = false;
+            auto issue_pv = [&](long long t, bool first) -> bool {
+                const int b = (int)(t & 1);
+                if (!wt.wait(smem_addr(&bars.p_full[b]), (uint32_t)((t >> 1) & 1))) return false;
+                if (first && vseg > 0 && !wt.wait(smem_addr(&bars.o_free), (uint32_t)((vseg - 1) & 1))) return false;
+                tc_fence_after();
+                const uint32_t sb = stage0 + (int)(t % NST) * C::kStageBytes;
+                const uint32_t pa = p_addr + b * C::kPBytes;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(pa + kk * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(sb + kk * 2048, C::kChunk, 1024);
+                    mma_ss(tmem + C::kColO, ad, bd, vexact ? C::kIdescPVf16 : C::kIdescPVbf16,
+                           (first && kk == 0) ? 0u : 1u);
+                }
+                mma_commit(smem_addr(&bars.empty[(int)(t % NST)]));
+                mma_commit(smem_addr(&bars.o_done[b]));
+                return true;
+            };
+            if (ok && n > 0) ok = issue_qk(0);
+            for (long long j = 0; ok && j < n; ++j) {
+                const SegFlags f = seg_flags(lo + j, lo, hi, vpos);
+                if (f.begin) {
+                    ++vseg;
+                    vexact = vpos.T < kExactPVBelow;
+                }
+                // within a segment QK^T(j+1) goes first; at a segment end PV(j) must go first,
+                // because the next segment's query load waits for the epilogue of this one
+                const bool next_same = j + 1 < n && !f.end;
+                if (next_same && !(ok = issue_qk(j + 1))) break;
+                if (!(ok = issue_pv(j, f.begin))) break;
+                if (!next_same && j + 1 < n && !(ok = issue_qk(j + 1))) break;
+                advance_unit(vpos, seq_lens, p.B, p.max_pages, p.gc);
             }
             // drain every MMA this thread issued before tensor memory is freed
             mma_commit(smem_addr(&bars.drain));
@@ -261,120 +349,137 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax / epilogue (warps 2..5)
+        // ------------------------------------------------------------ softmax / epilogue (warps 2..9)
+        const int sw = warp - kSoftmaxWarp0;              // 0..7
+        const int wg = sw >> 2;                           // which half of the tile columns and of O
         const int quad = warp & 3;
         const int row = quad * 32 + lane;                 // head row == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         const bool warp_active = quad * 32 < p.H;
         const bool row_active = row < p.H;
-        const int tid_sm = threadIdx.x - kSoftmaxWarp0 * 32;   // 0..127
+        const int tid_sm = threadIdx.x - kSoftmaxWarp0 * 32;   // 0..255
+        const float sc = p.scale_log2;
+        constexpr int kOHalf = LS / 2;                    // O columns per warpgroup
         UnitPos pos = pos0;
-        long long j = 0;
-        long long last_o = -1;                            // last PV whose completion was observed
-        float m = -INFINITY, l = 0.f;
+        long long last_o = -1;                            // highest PV index whose completion was observed
+        int seg = -1;
+        float m = -INFINITY, l = 0.f;                     // l: this warpgroup's half of the row sum
         bool first_tile = true;
+        bool exact = false;                               // fp16 PV for this segment
+        // PV(t) completes on o_done[t & 1]; completions are in order, so observing PV(t) covers all before it
         auto wait_o = [&](long long t) -> bool {
             if (t <= last_o) return true;
-            if (!wt.wait(smem_addr(&bars.o_done), (uint32_t)(t & 1))) return false;
+            if (!wt.wait(smem_addr(&bars.o_done[t & 1]), (uint32_t)((t >> 1) & 1))) return false;
             last_o = t;
             tc_fence_after();
             return true;
         };
-        for (long long u = lo; u < hi; ++u, ++j) {
-            const SegFlags f = seg_flags(u, lo, hi, pos);
+        long long j = 0;
+        for (; j < n; ++j) {
+            const SegFlags f = seg_flags(lo + j, lo, hi, pos);
             const int shard = p.shard0 + pos.s;
+            const int buf = (int)(j & 1);
             if (f.begin) {
-                // Q row of this head for (b, shard) into tensor memory: [q~_s | q_pe] as bf16 pairs
+                ++seg;
+                // query of this (b, shard): the latent part into tensor memory as bf16 pairs
+                // (warpgroups take alternate 64-element chunks), the RoPE part into shared memory
                 if (warp_active) {
                     const uint4* qs = reinterpret_cast<const uint4*>(q + ((size_t)pos.b * p.H + row) * p.L +
                                                                      (size_t)shard * LS);
-                    const uint4* qp = reinterpret_cast<const uint4*>(q_pe + ((size_t)pos.b * p.H + row) * RD);
 #pragma unroll
-                    for (int c = 0; c < C::kK / 64; ++c) {
+                    for (int c = wg; c < C::kChunksC; c += 2) {
                         uint32_t r[32];
 #pragma unroll
                         for (int v = 0; v < 8; ++v) {
                             uint4 x = make_uint4(0, 0, 0, 0);
-                            if (row_active) x = c < C::kChunksC ? __ldg(qs + c * 8 + v) : __ldg(qp + (c - C::kChunksC) * 8 + v);
+                            if (row_active) x = __ldg(qs + c * 8 + v);
                             r[4 * v + 0] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
                         }
                         tmem_st32(lane_base + C::kColQ + c * 32, r);
                     }
                     tmem_wait_st();
                 }
-                (void)effective_len(seq_lens, pos.b, p.max_pages, p.status);
+                {
+                    const uint4* qp = reinterpret_cast<const uint4*>(q_pe + ((size_t)pos.b * p.H + row) * RD);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int c = wg * 4 + k;
+                        const uint4 x = row_active ? __ldg(qp + c) : make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(qpe_smem + sw128_offset(row, c)) = x;
+                    }
+                    fence_proxy_async_smem();
+                }
+                if (wg == 0 && lane == 0) (void)effective_len(seq_lens, pos.b, p.max_pages, p.status);
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&bars.q_full));
+                warp_arrive(smem_addr(&bars.q_full));
                 m = -INFINITY;
                 l = 0.f;
                 first_tile = true;
+                exact = pos.T < kExactPVBelow;
             }
             const int valid = min(kPage, pos.T - pos.tile * kPage);
-            if (!wt.wait(smem_addr(&bars.s_full), (uint32_t)(j & 1))) break;
+            const bool tail = valid < kPage;
+            if (!wt.wait(smem_addr(&bars.s_full[buf]), (uint32_t)((j >> 1) & 1))) break;
             tc_fence_after();
-            float s[64];
-            if (warp_active) {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(lane_base + C::kColS, r0);
-                tmem_ld32(lane_base + C::kColS + 32, r1);
-                tmem_wait_ld();
-#pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    s[t] = __uint_as_float(r0[t]);
-                    s[t + 32] = __uint_as_float(r1[t]);
-                }
-            }
+            uint32_t sraw[32];
+            if (warp_active) tmem_ld32(lane_base + C::kColS + buf * 64 + wg * 32, sraw);
+            uint8_t* sb = smem + (int)(j % NST) * C::kStageBytes;
+            if (warp_active) tmem_wait_ld();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&bars.s_free));
+            warp_arrive(smem_addr(&bars.s_free[buf]));
 
-            // QK^T of this tile is done with its shared memory: turn the latent rows into the fp16
-            // operand of PV, and zero rows past the sequence end so P*C never meets stale bits
-            {
-                uint8_t* sb = smem + (int)(j % NST) * C::kStageBytes;
-#pragma unroll 4
-                for (int i = tid_sm; i < C::kChunksC * kPage * 8; i += 128) {
-                    const int c = i >> 9, rr = (i >> 3) & 63, seg16 = i & 7;
-                    uint4* ptr = reinterpret_cast<uint4*>(sb + c * C::kChunk + rr * 128 + seg16 * 16);
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (rr < valid) {
-                        v = *ptr;
-                        v.x = bf16x2_to_f16x2(v.x);
-                        v.y = bf16x2_to_f16x2(v.y);
-                        v.z = bf16x2_to_f16x2(v.z);
-                        v.w = bf16x2_to_f16x2(v.w);
+            // row extreme of the raw scores over this warpgroup's 32 columns
+            // (the maximum of scale * s is scale * max(s) for scale >= 0, scale * min(s) otherwise)
+            float s[32];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) s[t] = __uint_as_float(sraw[t]);
+            float ext = sc >= 0.f ? -INFINITY : INFINITY;
+            if (warp_active) {
+                if (!tail) {
+                    float e4[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) e4[k] = s[k];
+                    if (sc >= 0.f) {
+#pragma unroll
+                        for (int t = 4; t < 32; ++t) e4[t & 3] = fmaxf(e4[t & 3], s[t]);
+                        ext = fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]));
+                    } else {
+#pragma unroll
+                        for (int t = 4; t < 32; ++t) e4[t & 3] = fminf(e4[t & 3], s[t]);
+                        ext = fminf(fminf(e4[0], e4[1]), fminf(e4[2], e4[3]));
                     }
-                    *ptr = v;
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 32; ++t)
+                        if (wg * 32 + t < valid) ext = sc >= 0.f ? fmaxf(ext, s[t]) : fminf(ext, s[t]);
                 }
-                fence_proxy_async_smem();
             }
+            bars.xmax_buf[j & 1][wg][row] = ext;
+            warp_arrive(smem_addr(&bars.xmax));
+            if (!wt.wait(smem_addr(&bars.xmax), (uint32_t)(j & 1))) break;
+            const float other = bars.xmax_buf[j & 1][wg ^ 1][row];
+            const float mt = (sc >= 0.f ? fmaxf(ext, other) : fminf(ext, other)) * sc;   // max of scale*s
 
             bool alive = true;
             if (warp_active) {
-                float mt = -INFINITY;
-#pragma unroll
-                for (int t = 0; t < 64; ++t) {
-                    s[t] = t < valid ? s[t] * p.scale_log2 : -INFINITY;
-                    mt = fmaxf(mt, s[t]);
-                }
                 if (first_tile) {
                     m = mt;
                 } else {
                     const bool need = mt > m + kRescaleThreshold;
                     if (__any_sync(0xffffffffu, need)) {
                         const float m_use = need ? mt : m;
-                        const float alpha = exp2f(m - m_use);
-                        if (!wait_o(j - 1)) { alive = false; }
+                        const float alpha = ex2_approx(m - m_use);
+                        if (!wait_o(j - 1)) alive = false;
                         if (alive) {
 #pragma unroll 1
-                            for (int c = 0; c < LS / 32; ++c) {
+                            for (int c = 0; c < kOHalf / 32; ++c) {
+                                const uint32_t ta = lane_base + C::kColO + wg * kOHalf + c * 32;
                                 uint32_t r[32];
-                                tmem_ld32(lane_base + C::kColO + c * 32, r);
+                                tmem_ld32(ta, r);
                                 tmem_wait_ld();
 #pragma unroll
                                 for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-                                tmem_st32(lane_base + C::kColO + c * 32, r);
+                                tmem_st32(ta, r);
                             }
                             tmem_wait_st();
                             l *= alpha;
@@ -384,39 +489,87 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 }
             }
             if (!alive) break;
-            uint32_t pk[32];
+            uint32_t pk[16];
             if (warp_active) {
-                float ls = 0.f;
+                const float nm = -m;
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const float e0 = exp2f(s[2 * t] - m), e1 = exp2f(s[2 * t + 1] - m);
-                    ls += e0 + e1;
-                    pk[t] = pack_f16x2(e0, e1);
+                for (int t = 0; t < 32; ++t) s[t] = ex2_approx(fmaf(s[t], sc, nm));
+                if (tail) {
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) s[t] = wg * 32 + t < valid ? s[t] : 0.f;
                 }
-                l += ls;
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int t = 0; t < 32; ++t) l4[t & 3] += s[t];
+                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                if (exact) {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) pk[t] = pack_f16x2(s[2 * t], s[2 * t + 1]);
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(s[2 * t], s[2 * t + 1]);
+                }
+            } else {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) pk[t] = 0u;
             }
-            // the single P buffer is free once PV of the previous tile has completed
-            if (j > 0 && !wait_o(j - 1)) break;
-            if (warp_active) {
-                tmem_st32(lane_base + C::kColP, pk);
-                tmem_wait_st();
+            if (exact) {
+                // this tile's latent rows -> fp16 (rows past the sequence end -> 0) for PV;
+                // QK^T has finished reading them
+#pragma unroll
+                for (int k = 0; k < C::kCvt; ++k) {
+                    const int i = tid_sm + k * kSoftmaxWarps * 32;
+                    const int rr = (i >> 3) & 63;
+                    uint4* ptr = reinterpret_cast<uint4*>(sb + (i >> 9) * C::kChunk + rr * 128 + (i & 7) * 16);
+                    uint4 v = *ptr;
+                    if (rr < valid) {
+                        v.x = bf16x2_to_f16x2(v.x);
+                        v.y = bf16x2_to_f16x2(v.y);
+                        v.z = bf16x2_to_f16x2(v.z);
+                        v.w = bf16x2_to_f16x2(v.w);
+                    } else {
+                        v = make_uint4(0, 0, 0, 0);
+                    }
+                    *ptr = v;
+                }
+            } else if (tail) {
+                // bf16 tile kept as it is; only the rows past the sequence end are zeroed
+                const int rows = kPage - valid;
+                for (int i = tid_sm; i < C::kChunksC * rows * 8; i += kSoftmaxWarps * 32) {
+                    const int c = i / (rows * 8), rr = valid + (i / 8) % rows, seg16 = i % 8;
+                    *reinterpret_cast<uint4*>(sb + c * C::kChunk + rr * 128 + seg16 * 16) = make_uint4(0, 0, 0, 0);
+                }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&bars.p_full));
+            // P buffer `buf` is free once PV(j - 2), its last reader, has completed
+            if (j >= 2 && !wait_o(j - 2)) break;
+            {
+                uint8_t* pb = p_smem + buf * C::kPBytes;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    *reinterpret_cast<uint4*>(pb + sw128_offset(row, wg * 4 + k)) =
+                        make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+            }
+            fence_proxy_async_smem();
+            warp_arrive(smem_addr(&bars.p_full[buf]));
             first_tile = false;
 
             if (f.end) {
                 if (!wait_o(j)) break;
+                // the two warpgroups' halves of the softmax sum
+                bars.xsum_buf[seg & 1][wg][row] = l;
+                warp_arrive(smem_addr(&bars.xsum));
+                if (!wt.wait(smem_addr(&bars.xsum), (uint32_t)(seg & 1))) break;
+                const float lt = l + bars.xsum_buf[seg & 1][wg ^ 1][row];
+                const long long u = lo + j;
                 const long long seg_first = (u - pos.tile) < lo ? lo : (u - pos.tile);
                 const int slot = seg_first == lo ? w : p.W + pos.b * p.gc + pos.s;
                 if (warp_active) {
-                    const float inv_l = 1.0f / l;
-                    float4* dst = reinterpret_cast<float4*>(ws.part_o + ((size_t)slot * p.H + row) * LS);
+                    const float inv_l = 1.0f / lt;
+                    float4* dst = reinterpret_cast<float4*>(ws.part_o + ((size_t)slot * p.H + row) * LS + wg * kOHalf);
 #pragma unroll 1
-                    for (int c = 0; c < LS / 32; ++c) {
+                    for (int c = 0; c < kOHalf / 32; ++c) {
                         uint32_t r[32];
-                        tmem_ld32(lane_base + C::kColO + c * 32, r);
+                        tmem_ld32(lane_base + C::kColO + wg * kOHalf + c * 32, r);
                         tmem_wait_ld();
                         if (row_active) {
 #pragma unroll
@@ -427,11 +580,10 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                                                              __uint_as_float(r[4 * v + 3]) * inv_l);
                         }
                     }
-                    if (row_active) ws.part_lse[(size_t)slot * p.H + row] = m + log2f(l);
+                    if (row_active && wg == 0) ws.part_lse[(size_t)slot * p.H + row] = m + log2f(lt);
                 }
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&bars.o_free));
+                warp_arrive(smem_addr(&bars.o_free));
             }
             advance_unit(pos, seq_lens, p.B, p.max_pages, p.gc);
         }
@@ -485,11 +637,12 @@ cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16*
     CUtensorMap tc, tk;
     if (!make_map(&tc, ckv, LS, (uint64_t)p.num_pages * p.g * kPage)) return cudaErrorInvalidValue;
     if (!make_map(&tk, kpe, RD, (uint64_t)p.num_pages * kPage)) return cudaErrorInvalidValue;
-    const size_t smem = 1024 + (size_t)NST * C::kStageBytes + sizeof(Bars<NST>);
-    static_assert(C::kTmemCols < 512 || (1024 + NST * C::kStageBytes) > 116 * 1024,
-                  "a 512-column TMEM allocation needs one CTA per SM");
+    const size_t smem = C::kSmem + sizeof(Bars<NST>);
+    static_assert(C::kTmemCols < 512 || C::kSmem > 116 * 1024, "a 512-column TMEM allocation needs one CTA per SM");
+    static_assert(C::kSmem + sizeof(Bars<NST>) <= 227 * 1024, "shared memory");
     auto kern = attn_sm100_kernel<LS, RD, NST>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static unsigned long long attr_done = 0;
+    cudaError_t e = set_smem_once(kern, smem, &attr_done);
     if (e != cudaSuccess) return e;
     kern<<<p.W, kThreads, smem, stream>>>(tc, tk, p, q, q_pe, bt, seq_lens, ws, wait_ns, debug_stall);
     return cudaGetLastError();
@@ -507,9 +660,9 @@ cudaError_t launch_attention_sm100(const Plan& p, const __nv_bfloat16* q, const 
                                    int wait_limit_us, int debug_stall, cudaStream_t stream) {
     const uint64_t wait_ns = (wait_limit_us > 0 ? (uint64_t)wait_limit_us : 1000000ull) * 1000ull;
     switch (p.Ls) {
-        case 256: return launch_t<256, 64, 5>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
-        case 128: return launch_t<128, 64, 8>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
-        case 64: return launch_t<64, 64, 12>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
+        case 256: return launch_t<256, 64, 4>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
+        case 128: return launch_t<128, 64, 6>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
+        case 64: return launch_t<64, 64, 10>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
     }
     return cudaErrorNotSupported;
 }

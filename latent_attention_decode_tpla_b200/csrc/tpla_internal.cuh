@@ -158,6 +158,20 @@ __device__ inline void advance_unit(UnitPos& p, const int32_t* seq_lens, int B, 
     }
 }
 
+// Sets the dynamic shared-memory limit of `kern` once per device (a function
+// attribute; repeating it on every launch only costs host time).
+template <typename Kern>
+inline cudaError_t set_smem_once(Kern kern, size_t bytes, unsigned long long* done_mask) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) __atomic_fetch_or(done_mask, bit, __ATOMIC_RELEASE);
+    return e;
+}
+
 // ---------------------------------------------------------------- launchers (one per .cu file)
 
 cudaError_t launch_attention_simt(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16* q_pe,

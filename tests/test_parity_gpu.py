@@ -190,3 +190,14 @@ def test_mixed_b64_paged_with_append(kernel):
         got = hx.run_gpu(d_or, scale, mode=mode, shard=0, dev=dev, kernel=kernel)
         want = hx.run_oracle(d_or, scale, mode=mode, shard=0, batch=batch)
         hx.assert_close(got[batch], want, "mixed %s" % mode)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_pv_precision_modes_at_the_length_boundary(kernel):
+    """Sequences just below 8192 tokens run PV in fp16, from 8192 on in bf16; both meet the tolerance."""
+    d = _case(4, 128, 512, 64, 128, 2, [8191, 8192, 8193, 100], seed=23)
+    _kernel_or_skip(d, kernel)
+    scale = 1 / math.sqrt(192)
+    hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "all shards")
+    hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=1, kernel=kernel),
+                    hx.run_oracle(d, scale, mode="shard", shard=1), "shard 1")
