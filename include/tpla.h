@@ -156,6 +156,37 @@ int mla_decode(const tpla_dims_t* dims,
                void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * tpla_decode_static -- tpla_decode for callers that cannot allocate device
+ * memory and so cannot pass a workspace: code running inside a memory-pool or
+ * allocator callback, under a framework that owns all device memory, or in a
+ * loop where an allocation may block.  The TPLA paper has no counterpart;
+ * this is a property of this library only.
+ *
+ * Same arguments and result as tpla_decode, without workspace/ws_bytes.
+ * Its scratch is one file-scope device array of 32 MiB, which every GPU that
+ * loads the library holds until the process exits; the call allocates and
+ * frees nothing (no cudaMalloc, no allocating library routine).
+ *   - Size limit: the split-KV partials of B*g (sequence, shard) pairs plus at
+ *     least one worker must fit in 32 MiB, i.e. roughly
+ *     (B*g + 1) * H * (L/g) * 4 bytes plus a small header; larger problems
+ *     return TPLA_ERR_WORKSPACE with nothing enqueued.  Near the limit the
+ *     call uses fewer split-KV workers than tpla_decode (same result up to
+ *     fp32 rounding, possibly slower).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, once per device, with that device current);
+ *     make that first call before any stream capture.
+ *   - Every call on a device shares the one array, and it keeps the last
+ *     call's contents (nothing in it needs to start at zero).  Calls that
+ *     overlap on the GPU (different streams, or two host threads) race on
+ *     it: order them, e.g. on one stream.
+ */
+int tpla_decode_static(const tpla_dims_t* dims,
+                       const tpla_bf16* q_nope_absorbed, const tpla_bf16* q_pe,
+                       const tpla_bf16* ckv_cache, const tpla_bf16* kpe_cache,
+                       const int32_t* block_table, const int32_t* seq_lens,
+                       const tpla_bf16* w_uv, float* out, void* stream);
+
+/*
  * The two stages of a decode call, for callers that time or overlap them.
  * tpla_attention runs the split-KV attention of all shards (shard == -1) or
  * of one shard and leaves per-split partial outputs and log-sum-exps in

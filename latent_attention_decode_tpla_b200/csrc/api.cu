@@ -322,3 +322,79 @@ int tpla_get_option(int option) {
 const char* tpla_version(void) { return "tpla-b200 0.1 (sm_100a)"; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- decode without allocation
+//
+// For callers that cannot allocate device memory at all: code that runs where
+// cudaMalloc is off limits (inside a custom allocator or memory-pool callback,
+// under a framework that owns every byte of device memory and hands out
+// nothing, or in a hard real-time loop where an allocation may block), and
+// that therefore cannot provide a workspace.  tpla_decode_static does what
+// tpla_decode does with its scratch in one fixed, file-scope device array.
+namespace tpla {
+namespace {
+
+constexpr size_t kStaticScratchBytes = 32ull << 20;      // 32 MiB, held by every GPU that loads the library
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mutex;
+void* g_static_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per device
+// (the array's name in host code is only a host-side handle, not a device address).
+int static_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TPLA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return TPLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mutex);
+    if (!g_static_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || ptr == nullptr) return TPLA_ERR_CUDA;
+        g_static_ptr[dev] = ptr;
+    }
+    *out = g_static_ptr[dev];
+    return TPLA_OK;
+}
+
+}  // namespace
+}  // namespace tpla
+
+extern "C" int tpla_decode_static(const tpla_dims_t* dims, const tpla_bf16* q, const tpla_bf16* q_pe,
+                                  const tpla_bf16* ckv, const tpla_bf16* kpe, const int32_t* block_table,
+                                  const int32_t* seq_lens, const tpla_bf16* w_uv, float* out, void* stream) {
+    int st = check_dims(dims);
+    if (st) return st;
+    if (dims->B == 0) return TPLA_OK;
+    if (!q || !q_pe || !ckv || !kpe || !seq_lens || !out) return TPLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(q_pe) || !aligned16(ckv) || !aligned16(kpe) || !aligned16(seq_lens))
+        return TPLA_ERR_INVALID_ARG;
+    if (block_table && !aligned16(block_table)) return TPLA_ERR_INVALID_ARG;
+    if (w_uv && !aligned16(w_uv)) return TPLA_ERR_INVALID_ARG;
+    if (!block_table && (long long)dims->B * dims->max_pages_per_seq > dims->num_pages) return TPLA_ERR_INVALID_ARG;
+    // partial slots that fit next to the header and the log-sum-exp block
+    const size_t head = 256 + ws_lse_bytes(dims);
+    if (head >= kStaticScratchBytes) return TPLA_ERR_WORKSPACE;
+    const size_t slot_bytes = (size_t)dims->H * (size_t)(dims->L / dims->g) * sizeof(float);
+    const long long max_slots = (long long)((kStaticScratchBytes - head) / slot_bytes);
+    const long long fixed = (long long)dims->B * dims->g;          // one slot per (sequence, shard)
+    if (max_slots - fixed < 1) return TPLA_ERR_WORKSPACE;          // beyond the static scratch, even with one worker
+    void* scratch = nullptr;
+    if ((st = static_scratch(&scratch))) return st;
+    Plan p;
+    if ((st = make_plan(dims, -1, &p))) return st;
+    if (p.W > max_slots - fixed) p.W = (int)(max_slots - fixed);  // fewer split-KV workers, same result
+    Workspace w = carve(scratch, dims);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto bq = reinterpret_cast<const __nv_bfloat16*>(q);
+    auto bqp = reinterpret_cast<const __nv_bfloat16*>(q_pe);
+    auto bc = reinterpret_cast<const __nv_bfloat16*>(ckv);
+    auto bk = reinterpret_cast<const __nv_bfloat16*>(kpe);
+    cudaError_t e = sm100_supports(p) && g_opt_kernel != 1
+                        ? launch_attention_sm100(p, bq, bqp, bc, bk, block_table, seq_lens, w, g_opt_wait_limit,
+                                                 g_opt_debug_stall, s)
+                        : launch_attention_simt(p, bq, bqp, bc, bk, block_table, seq_lens, w, s);
+    if (e == cudaErrorNotSupported) return TPLA_ERR_UNSUPPORTED;
+    if (e != cudaSuccess) return TPLA_ERR_CUDA;
+    e = launch_combine(p, seq_lens, reinterpret_cast<const __nv_bfloat16*>(w_uv), out, w, s);
+    return e == cudaSuccess ? TPLA_OK : TPLA_ERR_CUDA;
+}

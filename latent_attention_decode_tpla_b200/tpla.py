@@ -37,7 +37,8 @@ PAGE_SIZE = 64
 
 EXPORTED = ("tpla_status_string", "tpla_decode_workspace_size", "tpla_decode", "tpla_decode_shard",
             "mla_decode", "tpla_attention", "tpla_combine", "tpla_append_kv",
-            "tpla_check_device_status", "tpla_set_option", "tpla_get_option", "tpla_version")
+            "tpla_check_device_status", "tpla_set_option", "tpla_get_option", "tpla_version",
+            "tpla_decode_static")
 
 
 class Dims(ctypes.Structure):
@@ -87,6 +88,7 @@ def lib():
             "tpla_set_option": ([_I, _I], _I),
             "tpla_get_option": ([_I], _I),
             "tpla_version": ([], ctypes.c_char_p),
+            "tpla_decode_static": ([_DIMS, _P, _P, _P, _P, _P, _P, _P, _P, _P], _I),
         }
         for name, (args, res) in sigs.items():
             f = getattr(L, name)
@@ -174,6 +176,14 @@ def mla_decode(dims, q, q_pe, ckv, kpe, block_table, seq_lens, w_uv, out, worksp
     _check(lib().mla_decode(ctypes.byref(dims), _bf16(q), _bf16(q_pe), _bf16(ckv), _bf16(kpe),
                             _i32(block_table), _i32(seq_lens), _bf16(w_uv), _f32(out), _ptr(workspace),
                             workspace.numel(), _stream(stream)), "mla_decode")
+    return out
+
+
+def decode_static(dims, q, q_pe, ckv, kpe, block_table, seq_lens, w_uv, out, stream=None):
+    """tpla_decode without a workspace: scratch is the library's fixed 32 MiB device array."""
+    _check(lib().tpla_decode_static(ctypes.byref(dims), _bf16(q), _bf16(q_pe), _bf16(ckv), _bf16(kpe),
+                                    _i32(block_table), _i32(seq_lens), _bf16(w_uv), _f32(out), _stream(stream)),
+           "tpla_decode_static")
     return out
 
 
