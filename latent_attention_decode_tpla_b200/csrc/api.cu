@@ -56,9 +56,19 @@ size_t ws_lse_bytes(const tpla_dims_t* d) {
     return align_up((size_t)(kMaxWorkers + (size_t)d->B * d->g) * d->H * sizeof(float), 256);
 }
 
+// Workspace: 256-byte header | log-sum-exps [kMaxWorkers + B*g][H] | partial outputs [slots][H][L/g]
+// | merged shard outputs [B][H][L].  `slots` is kMaxWorkers + B*g for a caller's workspace.
+size_t ws_part_bytes(const tpla_dims_t* d, size_t slots) {
+    return align_up(slots * d->H * (size_t)(d->L / d->g) * sizeof(float), 256);
+}
+
+size_t ws_merged_bytes(const tpla_dims_t* d) {
+    return align_up((size_t)d->B * d->H * d->L * sizeof(float), 256);
+}
+
 size_t ws_bytes_for(const tpla_dims_t* d) {
     const size_t slots = (size_t)kMaxWorkers + (size_t)d->B * d->g;
-    return 256 + ws_lse_bytes(d) + slots * d->H * (size_t)(d->L / d->g) * sizeof(float);
+    return 256 + ws_lse_bytes(d) + ws_part_bytes(d, slots) + ws_merged_bytes(d);
 }
 
 int device_info(unsigned** status, int* sms) {
@@ -118,11 +128,13 @@ int make_plan(const tpla_dims_t* d, int shard, Plan* p) {
     return TPLA_OK;
 }
 
-Workspace carve(void* workspace, const tpla_dims_t* d) {
+Workspace carve(void* workspace, const tpla_dims_t* d, size_t slots = 0) {
+    if (slots == 0) slots = (size_t)kMaxWorkers + (size_t)d->B * d->g;
     char* base = static_cast<char*>(workspace) + 256;
     Workspace w;
     w.part_lse = reinterpret_cast<float*>(base);
     w.part_o = reinterpret_cast<float*>(base + ws_lse_bytes(d));
+    w.merged = reinterpret_cast<float*>(base + ws_lse_bytes(d) + ws_part_bytes(d, slots));
     return w;
 }
 
@@ -160,7 +172,7 @@ int run_combine(const tpla_dims_t* d, int shard, const int32_t* seq_lens, const 
     if (st) return st;
     if (shard < -1 || shard >= d->g) return TPLA_ERR_INVALID_ARG;
     if (d->B == 0) return TPLA_OK;
-    if (!seq_lens || !out) return TPLA_ERR_INVALID_ARG;
+    if (!seq_lens || !out || !aligned16(out)) return TPLA_ERR_INVALID_ARG;
     if (w_uv && !aligned16(w_uv)) return TPLA_ERR_INVALID_ARG;
     if (!workspace || !aligned16(workspace)) return TPLA_ERR_WORKSPACE;
     if (ws_bytes < ws_bytes_for(d)) return TPLA_ERR_WORKSPACE;
@@ -177,7 +189,7 @@ int run_decode(const tpla_dims_t* d, int shard, const tpla_bf16* q, const tpla_b
                size_t ws_bytes, void* stream) {
     int st = check_decode(d, shard, q, q_pe, ckv, kpe, block_table, seq_lens, workspace, ws_bytes);
     if (st) return st;
-    if (d->B > 0 && !out) return TPLA_ERR_INVALID_ARG;
+    if (d->B > 0 && (!out || !aligned16(out))) return TPLA_ERR_INVALID_ARG;
     if (w_uv && !aligned16(w_uv)) return TPLA_ERR_INVALID_ARG;
     if ((st = run_attention(d, shard, q, q_pe, ckv, kpe, block_table, seq_lens, workspace, ws_bytes, stream)))
         return st;
@@ -366,13 +378,14 @@ extern "C" int tpla_decode_static(const tpla_dims_t* dims, const tpla_bf16* q, c
     if (st) return st;
     if (dims->B == 0) return TPLA_OK;
     if (!q || !q_pe || !ckv || !kpe || !seq_lens || !out) return TPLA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(q_pe) || !aligned16(ckv) || !aligned16(kpe) || !aligned16(seq_lens))
+    if (!aligned16(q) || !aligned16(q_pe) || !aligned16(ckv) || !aligned16(kpe) || !aligned16(seq_lens) ||
+        !aligned16(out))
         return TPLA_ERR_INVALID_ARG;
     if (block_table && !aligned16(block_table)) return TPLA_ERR_INVALID_ARG;
     if (w_uv && !aligned16(w_uv)) return TPLA_ERR_INVALID_ARG;
     if (!block_table && (long long)dims->B * dims->max_pages_per_seq > dims->num_pages) return TPLA_ERR_INVALID_ARG;
-    // partial slots that fit next to the header and the log-sum-exp block
-    const size_t head = 256 + ws_lse_bytes(dims);
+    // partial slots that fit next to the header, the log-sum-exp block and the merged outputs
+    const size_t head = 256 + ws_lse_bytes(dims) + ws_merged_bytes(dims) + 256;
     if (head >= kStaticScratchBytes) return TPLA_ERR_WORKSPACE;
     const size_t slot_bytes = (size_t)dims->H * (size_t)(dims->L / dims->g) * sizeof(float);
     const long long max_slots = (long long)((kStaticScratchBytes - head) / slot_bytes);
@@ -383,7 +396,7 @@ extern "C" int tpla_decode_static(const tpla_dims_t* dims, const tpla_bf16* q, c
     Plan p;
     if ((st = make_plan(dims, -1, &p))) return st;
     if (p.W > max_slots - fixed) p.W = (int)(max_slots - fixed);  // fewer split-KV workers, same result
-    Workspace w = carve(scratch, dims);
+    Workspace w = carve(scratch, dims, (size_t)p.W + (size_t)fixed);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     auto bq = reinterpret_cast<const __nv_bfloat16*>(q);
     auto bqp = reinterpret_cast<const __nv_bfloat16*>(q_pe);

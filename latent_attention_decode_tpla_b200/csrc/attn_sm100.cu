@@ -322,20 +322,53 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 mma_commit(smem_addr(&bars.o_done[b]));
                 return true;
             };
-            if (ok && n > 0) ok = issue_qk(0);
-            for (long long j = 0; ok && j < n; ++j) {
-                const SegFlags f = seg_flags(lo + j, lo, hi, vpos);
-                if (f.begin) {
-                    ++vseg;
-                    vexact = vpos.T < kExactPVBelow;
+            // Issue whichever MMA is ready, polling without blocking: QK^T of the next tile as
+            // soon as its stage has landed and its S buffer is free, PV of the oldest tile as
+            // soon as its P is in shared memory.  Neither stream waits on the other.
+            long long jq = 0, jv = 0;
+            bool vbegun = false;
+            long long idle_since = clock64();
+            while (ok && jv < n) {
+                bool did = false;
+                if (jq < n) {
+                    const SegFlags fq = seg_flags(lo + jq, lo, hi, qpos);
+                    const int st = (int)(jq % NST), b = (int)(jq & 1);
+                    if ((!fq.begin || mbar_test_wait(smem_addr(&bars.q_full), (uint32_t)((qseg + 1) & 1))) &&
+                        mbar_test_wait(smem_addr(&bars.full[st]), (uint32_t)((jq / NST) & 1)) &&
+                        (jq < 2 || mbar_test_wait(smem_addr(&bars.s_free[b]), (uint32_t)(((jq >> 1) - 1) & 1)))) {
+                        ok = issue_qk(jq);       // its waits are already satisfied
+                        ++jq;
+                        did = true;
+                    }
                 }
-                // within a segment QK^T(j+1) goes first; at a segment end PV(j) must go first,
-                // because the next segment's query load waits for the epilogue of this one
-                const bool next_same = j + 1 < n && !f.end;
-                if (next_same && !(ok = issue_qk(j + 1))) break;
-                if (!(ok = issue_pv(j, f.begin))) break;
-                if (!next_same && j + 1 < n && !(ok = issue_qk(j + 1))) break;
-                advance_unit(vpos, seq_lens, p.B, p.max_pages, p.gc);
+                if (ok && jv < jq) {
+                    const SegFlags fv = seg_flags(lo + jv, lo, hi, vpos);
+                    if (fv.begin && !vbegun) {
+                        ++vseg;
+                        vexact = vpos.T < kExactPVBelow;
+                        vbegun = true;
+                    }
+                    const int b = (int)(jv & 1);
+                    if (mbar_test_wait(smem_addr(&bars.p_full[b]), (uint32_t)((jv >> 1) & 1)) &&
+                        (!fv.begin || vseg == 0 ||
+                         mbar_test_wait(smem_addr(&bars.o_free), (uint32_t)((vseg - 1) & 1)))) {
+                        ok = issue_pv(jv, fv.begin);
+                        advance_unit(vpos, seq_lens, p.B, p.max_pages, p.gc);
+                        ++jv;
+                        vbegun = false;
+                        did = true;
+                    }
+                }
+                if (did) {
+                    idle_since = clock64();
+                } else {
+                    if (bars.abort) break;
+                    if ((uint64_t)(clock64() - idle_since) > wt.limit_cycles) {
+                        atomicOr(p.status, kStatusTimeout);
+                        bars.abort = 1;
+                        break;
+                    }
+                }
             }
             // drain every MMA this thread issued before tensor memory is freed
             mma_commit(smem_addr(&bars.drain));
@@ -492,8 +525,10 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             uint32_t pk[16];
             if (warp_active) {
                 const float nm = -m;
+                // even columns on the special-function unit, odd columns on the FMA pipe
 #pragma unroll
-                for (int t = 0; t < 32; ++t) s[t] = ex2_approx(fmaf(s[t], sc, nm));
+                for (int t = 0; t < 32; ++t)
+                    s[t] = (t & 1) ? ex2_fma(fmaf(s[t], sc, nm)) : ex2_approx(fmaf(s[t], sc, nm));
                 if (tail) {
 #pragma unroll
                     for (int t = 0; t < 32; ++t) s[t] = wg * 32 + t < valid ? s[t] : 0.f;

@@ -52,6 +52,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// non-blocking test of a phase (returns at once)
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int x, int y) {
@@ -160,6 +173,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA and integer pipes, for x <= 0 (the special-function unit is the
+// softmax's bottleneck, so part of the exponentials are computed here instead).
+// Range reduction x = i + f with i = round(x) (adding 1.5 * 2^23 rounds x to an
+// integer held in the low mantissa bits) and f in [-0.5, 0.5]; 2^f by a
+// degree-4 polynomial fitted to 2^f on that interval for least maximum relative
+// error (2.7e-6, well under the 16-bit rounding of P that follows); 2^i is added
+// to the exponent field.  Inputs below -120 are clamped (2^-120 is zero at the
+// precision that matters here).
+__device__ __forceinline__ float ex2_fma(float x) {
+    x = fmaxf(x, -120.0f);
+    const float t = x + 12582912.0f;
+    const float f = x - (t - 12582912.0f);
+    float y = fmaf(0.009570068679749966f, f, 0.055917806923389435f);
+    y = fmaf(y, f, 0.240247443318367f);
+    y = fmaf(y, f, 0.6931218504905701f);
+    y = fmaf(y, f, 0.9999992847442627f);
+    return __int_as_float(__float_as_int(y) + (__float_as_int(t) << 23));
 }
 
 // ------------------------------------------------------------------ descriptors
