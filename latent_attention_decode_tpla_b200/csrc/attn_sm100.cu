@@ -5,29 +5,30 @@
 // for every shard s of sequence b and every head h
 //     z_t = scale * (q~_h[s-slice] . c_{t,s} + q_pe_h . k_pe_t)
 //     o_{h,s} = sum_t softmax_t(z) c_{t,s}
-// as an online softmax over 64-token tiles of one split-KV segment
-// (schedule in tpla_internal.cuh); the result per segment is the normalised
-// o and log2-sum-exp per head, merged later by the combine kernel.
+// as an online softmax over the tiles of one split-KV segment (schedule in
+// tpla_internal.cuh); the result per segment is the normalised o and the
+// log2-sum-exp per head, merged later by the combine kernels.
 //
 // All heads of a sequence share every cache row, so both contractions are
 // dense with the heads as the MMA M dimension (M = 128; fewer heads are
-// padded):
-//     S[h, t]  = Q[h, :] . [C_s | K_pe][t, :]^T     M=128, N=64,  K=Ls+R
-//     O[h, :] += P[h, t] . C_s[t, :]                M=128, N=Ls,  K=64
-// One 64-token tile is TMA-loaded once into 128B-swizzled shared memory and
-// is the K-major B operand of the first MMA and the MN-major B operand of
-// the second.
+// padded).  A tile is two consecutive 64-token pages of one segment (one page
+// where a segment has an odd number of pages left; the other half is then
+// zero-filled by TMA and masked):
+//     S[h, t]  = Q[h, :] . [C_s | K_pe][t, :]^T     M=128, N=128, K=Ls+R
+//     O[h, :] += P[h, t] . C_s[t, :]                M=128, N=Ls,  K=128
+// N = 128 matters: on B200 a 128x64x16 MMA takes about as long as a
+// 128x128x16 one, so 64-token tiles spend twice the tensor time on QK^T.
+// The tile is TMA-loaded once into 128B-swizzled shared memory, each 16 KB
+// chunk holding one 64-column slice of both pages (rows 0-63 the first page,
+// rows 64-127 the second), and it is the K-major B operand of QK^T and the
+// MN-major B operand of PV.
 //
 // Operand placement (tensor memory holds 512 columns of 128 lanes):
-//   tensor memory: O (Ls columns, fp32), two S buffers (64 columns each,
-//                  fp32), and the latent part of Q (Ls/2 columns, bf16
-//                  pairs) as the A operand of the first Ls/16 QK^T steps;
-//   shared memory: the RoPE part of Q (A operand of the last R/16 QK^T
-//                  steps) and two P buffers (A operand of PV), all in the
-//                  128B-swizzled K-major layout.
-// With two S and two P buffers the MMA warp issues QK^T(j+1) before PV(j):
-// the softmax of tile j has the time of PV(j-1) + QK^T(j+1) to produce P(j)
-// before the tensor pipe needs it.
+//   tensor memory: O (Ls columns, fp32), S (128 columns, fp32) and the latent
+//                  part of Q (Ls/2 columns, bf16 pairs) as the A operand of
+//                  the first Ls/16 QK^T steps;
+//   shared memory: the RoPE part of Q (A operand of the last R/16 QK^T steps)
+//                  and P (A operand of PV), in the 128B-swizzled K-major layout.
 //
 // Precision: QK^T multiplies the bf16 inputs as they are.  PV multiplies the
 // probabilities P, rounded to 16 bits, by the latent tile.  Rounding P to
@@ -42,22 +43,26 @@
 // unless its magnitude is below 2^-14).  Longer sequences keep the bf16 tile
 // and bf16 P, which costs no extra shared-memory traffic.  In both modes the
 // rows past the end of the sequence are zeroed before PV reads the tile.
+// All exponentials run on the special-function unit: moving a share of them
+// to a polynomial on the FMA pipe measured slower here, since the softmax is
+// bound by its latency chain, not by that unit's throughput.
 //
 // Warp roles (320 threads): warp 0 issues TMA loads into a ring of NST
-// stages (page-table entries fetched a few tiles ahead); warp 1 allocates
-// tensor memory and issues the MMAs (one thread); warps 2-9 are two softmax
+// stages (page-table entries fetched a few pages ahead); warp 1 allocates
+// tensor memory and issues the MMAs from one thread, polling for whichever
+// of QK^T(next tile) and PV(oldest tile) is ready; warps 2-9 are two softmax
 // warpgroups.  Both own all 128 TMEM lanes (one head row per thread);
-// warpgroup 0 takes score columns 0-31 of every tile, warpgroup 1 columns
-// 32-63, and they agree on each row's running maximum through a per-tile
+// warpgroup 0 takes score columns 0-63 of every tile, warpgroup 1 columns
+// 64-127, and they agree on each row's running maximum through a per-tile
 // exchange.  Each warpgroup rescales, and finally writes, its half of the O
 // columns.  O is rescaled only when a row's running maximum grows by more
 // than 8 (log2 units); a stale maximum only bounds p by 2^8.
 //
-// Every wait is bounded in time (SM clock cycles); a wait that runs out records
-// TPLA_ERR_TIMEOUT in the device status word, sets a CTA-wide abort flag so
-// all roles stop, and the kernel drains its TMA loads and MMAs before it
-// frees tensor memory and returns.  No role waits on a plain CTA barrier
-// while another may have stopped.
+// Every wait is bounded in time (SM clock cycles); a wait that runs out
+// records TPLA_ERR_TIMEOUT in the device status word, sets a CTA-wide abort
+// flag so all roles stop, and the kernel drains its TMA loads and MMAs
+// before it frees tensor memory and returns.  No role waits on a plain CTA
+// barrier while another may have stopped.
 #include "tpla_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -72,39 +77,41 @@ using namespace sm100;
 constexpr int kThreads = 320;
 constexpr int kSoftmaxWarp0 = 2;
 constexpr int kSoftmaxWarps = 8;
+constexpr int kTileTok = 2 * kPage;           // tokens per tile: two pages
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 constexpr int kExactPVBelow = 8192;           // sequences shorter than this run PV in fp16
 constexpr int kPageAhead = 4;                 // page-table entries the producer loads ahead
 
 template <int LS, int RD, int NST>
 struct Cfg {
-    static constexpr int kChunk = 64 * 128;                   // one 64-row x 128-byte swizzled chunk
+    static constexpr int kChunk = kTileTok * 128;             // 128 rows x 128 bytes: both pages of a 64-column slice
+    static constexpr int kHalf = kPage * 128;                  // one page's 64 rows of a chunk
     static constexpr int kChunksC = LS / 64;
     static constexpr int kStageBytes = (kChunksC + 1) * kChunk;   // latent chunks + the RoPE chunk
-    static constexpr int kPBytes = 128 * 128;                  // one P buffer: 128 rows x 64 tokens x 2 B
+    static constexpr int kPChunk = 128 * 128;                  // P: 128 rows x 64 tokens x 2 B, two of them
     static constexpr int kQpeBytes = 128 * 128;                // RoPE query: 128 rows x 64 x 2 B
     static constexpr int kColO = 0;
-    static constexpr int kColS = LS;                           // two buffers of 64 columns
-    static constexpr int kColQ = LS + 128;                     // latent query, LS/2 columns
+    static constexpr int kColS = LS;                           // 128 columns
+    static constexpr int kColQ = LS + kTileTok;                // latent query, LS/2 columns
     static constexpr int kColsUsed = kColQ + LS / 2;
     static constexpr int kTmemCols = kColsUsed <= 128 ? 128 : (kColsUsed <= 256 ? 256 : 512);
     static constexpr int kStepsC = LS / 16;                    // QK^T steps over the latent
     static constexpr int kStepsR = RD / 16;                    // QK^T steps over the RoPE key
-    static constexpr uint32_t kIdescQK = idesc_f16kind(128, 64, false, true);    // bf16 x bf16
-    static constexpr uint32_t kIdescPVf16 = idesc_f16kind(128, LS, true, false);  // fp16 x fp16
-    static constexpr uint32_t kIdescPVbf16 = idesc_f16kind(128, LS, true, true);  // bf16 x bf16
-    static constexpr int kCvt = kChunksC * kPage * 8 / (kSoftmaxWarps * 32);      // 16-byte pieces per thread
-    static constexpr size_t kSmem = 1024 + (size_t)NST * kStageBytes + 2 * kPBytes + kQpeBytes;
+    static constexpr uint32_t kIdescQK = idesc_f16kind(128, kTileTok, false, true);   // bf16 x bf16
+    static constexpr uint32_t kIdescPVf16 = idesc_f16kind(128, LS, true, false);       // fp16 x fp16
+    static constexpr uint32_t kIdescPVbf16 = idesc_f16kind(128, LS, true, true);       // bf16 x bf16
+    static constexpr int kCvt = kChunksC * kTileTok * 8 / (kSoftmaxWarps * 32);        // 16-byte pieces per thread
+    static constexpr size_t kSmem = 1024 + (size_t)NST * kStageBytes + 2 * kPChunk + kQpeBytes;
     static_assert(kColsUsed <= 512, "tensor memory");
     static_assert(LS % 64 == 0 && RD == 64, "tile shape");
-    static_assert(kCvt >= 1 && kChunksC * kPage * 8 % (kSoftmaxWarps * 32) == 0, "conversion split");
+    static_assert(kCvt >= 1 && kChunksC * kTileTok * 8 % (kSoftmaxWarps * 32) == 0, "conversion split");
 };
 
 template <int NST>
 struct Bars {
     uint64_t full[NST];
     uint64_t empty[NST];
-    uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+    uint64_t s_full, s_free, p_full, o_done;
     uint64_t q_full, o_free, xmax, xsum, drain, never;
     float xmax_buf[2][2][128];     // [tile parity][warpgroup][row]
     float xsum_buf[2][2][128];     // [segment parity][warpgroup][row]
@@ -134,12 +141,34 @@ struct Waiter {
     }
 };
 
-struct SegFlags {
-    bool begin, end;
+// A tile: one or two consecutive units (pages) of one (sequence, shard) segment.
+struct Tile {
+    UnitPos pos;      // first unit of the tile
+    long long u;      // its index in the unit order
+    int npages;       // 1 or 2
+    bool begin, end;  // first / last tile of its segment
 };
 
-__device__ __forceinline__ SegFlags seg_flags(long long u, long long lo, long long hi, const UnitPos& pos) {
-    return {u == lo || pos.tile == 0, u == hi - 1 || pos.tile == pos.ntiles - 1};
+__device__ __forceinline__ Tile make_tile(const UnitPos& pos, long long u, long long lo, long long hi) {
+    Tile t;
+    t.pos = pos;
+    t.u = u;
+    const long long left_seg = pos.ntiles - pos.tile;   // pages of this (b, s) from u on
+    const long long left_rng = hi - u;                 // units of the worker from u on
+    const long long left = left_seg < left_rng ? left_seg : left_rng;
+    t.npages = left >= 2 ? 2 : 1;
+    t.begin = u == lo || pos.tile == 0;
+    t.end = t.npages == left;
+    return t;
+}
+
+// the tile after `t`
+__device__ __forceinline__ Tile next_tile(const Tile& t, const int32_t* seq_lens, const Plan& p, long long lo,
+                                          long long hi) {
+    UnitPos pos = t.pos;
+    advance_unit(pos, seq_lens, p.B, p.max_pages, p.gc);
+    if (t.npages == 2) advance_unit(pos, seq_lens, p.B, p.max_pages, p.gc);
+    return make_tile(pos, t.u + t.npages, lo, hi);
 }
 
 // warp-collective: all lanes of the warp arrive through lane 0 after their prior writes
@@ -148,7 +177,7 @@ __device__ __forceinline__ void warp_arrive(uint32_t bar) {
     if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-// byte offset of 16-byte piece `c` of row `r` in a 128-row, 128B-swizzled K-major operand
+// byte offset of 16-byte piece `c` of row `r` in a 128B-swizzled K-major operand (rows of 128 bytes)
 __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
     return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
@@ -164,8 +193,8 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     // 1024-byte aligned base, by pointer arithmetic on the shared array so that every access
     // derived from it stays a shared-memory access
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    uint8_t* p_smem = smem + NST * C::kStageBytes;          // two P buffers
-    uint8_t* qpe_smem = p_smem + 2 * C::kPBytes;            // RoPE query
+    uint8_t* p_smem = smem + NST * C::kStageBytes;          // P: two K chunks of 64 tokens
+    uint8_t* qpe_smem = p_smem + 2 * C::kPChunk;            // RoPE query
     auto& bars = *reinterpret_cast<Bars<NST>*>(qpe_smem + C::kQpeBytes);
     const uint32_t stage0 = smem_addr(smem);
     const uint32_t p_addr = smem_addr(p_smem);
@@ -180,19 +209,16 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     const long long lo = unit_lo(w, U, p.W), hi = unit_lo(w + 1, U, p.W);
     if (lo >= hi) return;
     const UnitPos pos0 = warp_locate_unit(seq_lens, p.B, p.max_pages, p.gc, lo);
-    const long long n = hi - lo;                            // tiles of this worker
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) {
             mbar_init(smem_addr(&bars.full[i]), 1);
             mbar_init(smem_addr(&bars.empty[i]), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_addr(&bars.s_full[i]), 1);
-            mbar_init(smem_addr(&bars.s_free[i]), kSoftmaxWarps);
-            mbar_init(smem_addr(&bars.p_full[i]), kSoftmaxWarps);
-            mbar_init(smem_addr(&bars.o_done[i]), 1);
-        }
+        mbar_init(smem_addr(&bars.s_full), 1);
+        mbar_init(smem_addr(&bars.s_free), kSoftmaxWarps);
+        mbar_init(smem_addr(&bars.p_full), kSoftmaxWarps);
+        mbar_init(smem_addr(&bars.o_done), 1);
         mbar_init(smem_addr(&bars.q_full), kSoftmaxWarps);
         mbar_init(smem_addr(&bars.o_free), kSoftmaxWarps);
         mbar_init(smem_addr(&bars.xmax), kSoftmaxWarps);
@@ -217,45 +243,63 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            UnitPos pos = pos0;
             // page-table entries are loaded kPageAhead units ahead of their TMA issue
             UnitPos ahead = pos0;
+            long long ua = lo;
             int pg[kPageAhead];
 #pragma unroll
             for (int k = 0; k < kPageAhead; ++k) {
-                pg[k] = k < n ? page_lookup(block_table, ahead.b, ahead.tile, p.max_pages, p.num_pages, p.status) : -1;
-                if (k < n) advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
+                pg[k] = -1;
+                if (ua < hi) {
+                    pg[k] = page_lookup(block_table, ahead.b, ahead.tile, p.max_pages, p.num_pages, p.status);
+                    advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
+                    ++ua;
+                }
             }
-            long long j = 0;
-            for (; j < n; ++j) {
-                const int st = (int)(j % NST);
-                const uint32_t use = (uint32_t)(j / NST);
+            auto pop_page = [&]() -> int {
                 const int page = pg[0];
 #pragma unroll
                 for (int k = 0; k + 1 < kPageAhead; ++k) pg[k] = pg[k + 1];
-                if (j + kPageAhead < n) {
-                    pg[kPageAhead - 1] = page_lookup(block_table, ahead.b, ahead.tile, p.max_pages, p.num_pages, p.status);
+                pg[kPageAhead - 1] = -1;
+                if (ua < hi) {
+                    pg[kPageAhead - 1] =
+                        page_lookup(block_table, ahead.b, ahead.tile, p.max_pages, p.num_pages, p.status);
                     advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
+                    ++ua;
                 }
+                return page;
+            };
+            Tile t = make_tile(pos0, lo, lo, hi);
+            long long j = 0;
+            for (; t.u < hi; ++j) {
+                const int st = (int)(j % NST);
+                const uint32_t use = (uint32_t)(j / NST);
+                const int page0 = pop_page();
+                const int page1 = t.npages == 2 ? pop_page() : -1;
                 if (use > 0 && !wt.wait(smem_addr(&bars.empty[st]), (use - 1) & 1)) break;
-                const int shard = p.shard0 + pos.s;
-                // an invalid page reads rows past the end of the tensor: TMA fills zeros
-                const int yc = page >= 0 ? (page * p.g + shard) * kPage : p.num_pages * p.g * kPage;
-                const int yk = page >= 0 ? page * kPage : p.num_pages * kPage;
+                const int shard = p.shard0 + t.pos.s;
                 const uint32_t full = smem_addr(&bars.full[st]);
                 const uint32_t dst = stage0 + st * C::kStageBytes;
                 mbar_arrive_expect_tx(full, C::kStageBytes);
 #pragma unroll
-                for (int c = 0; c < C::kChunksC; ++c) tma_load_2d(dst + c * C::kChunk, &tm_c, full, c * 64, yc);
-                tma_load_2d(dst + C::kChunksC * C::kChunk, &tm_k, full, 0, yk);
-                advance_unit(pos, seq_lens, p.B, p.max_pages, p.gc);
+                for (int k = 0; k < 2; ++k) {
+                    // a missing or invalid page reads rows past the end of the tensor: TMA fills zeros
+                    const int page = k == 0 ? page0 : page1;
+                    const int yc = page >= 0 ? (page * p.g + shard) * kPage : p.num_pages * p.g * kPage;
+                    const int yk = page >= 0 ? page * kPage : p.num_pages * kPage;
+#pragma unroll
+                    for (int c = 0; c < C::kChunksC; ++c)
+                        tma_load_2d(dst + c * C::kChunk + k * C::kHalf, &tm_c, full, c * 64, yc);
+                    tma_load_2d(dst + C::kChunksC * C::kChunk + k * C::kHalf, &tm_k, full, 0, yk);
+                }
+                t = next_tile(t, seq_lens, p, lo, hi);
             }
             // drain: the last use of every stage must have landed before the CTA exits
-            for (long long t = j - NST < 0 ? 0 : j - NST; t < j; ++t) {
-                const int st = (int)(t % NST);
+            for (long long x = j - NST < 0 ? 0 : j - NST; x < j; ++x) {
+                const int st = (int)(x % NST);
                 // bounded wait that ignores the abort flag (the copy is in flight either way)
                 const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(smem_addr(&bars.full[st]), (uint32_t)(t / NST) & 1)) {
+                while (!mbar_try_wait(smem_addr(&bars.full[st]), (uint32_t)(x / NST) & 1)) {
                     if (globaltimer_ns() - t0 > wait_ns) {
                         atomicOr(p.status, kStatusTimeout);
                         break;
@@ -269,91 +313,65 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         if (lane == 0) {
             bool ok = true;
             if (debug_stall) ok = wt.wait(smem_addr(&bars.never), 0);   // nothing arrives: exercises the time-out
-            // QK^T runs one tile ahead of PV, each with its own cursor over the worker's tiles
-            UnitPos qpos = pos0;
-            int qseg = -1;
-            auto issue_qk = [&](long long t) -> bool {
-                const SegFlags f = seg_flags(lo + t, lo, hi, qpos);
-                if (f.begin) {
-                    ++qseg;
-                    if (!wt.wait(smem_addr(&bars.q_full), (uint32_t)(qseg & 1))) return false;
-                }
-                const int st = (int)(t % NST);
-                if (!wt.wait(smem_addr(&bars.full[st]), (uint32_t)((t / NST) & 1))) return false;
-                const int b = (int)(t & 1);
-                if (t >= 2 && !wt.wait(smem_addr(&bars.s_free[b]), (uint32_t)(((t >> 1) - 1) & 1))) return false;
-                tc_fence_after();
-                const uint32_t sb = stage0 + st * C::kStageBytes;
-                const uint32_t d = tmem + C::kColS + b * 64;
-#pragma unroll
-                for (int kk = 0; kk < C::kStepsC; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(sb + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024);
-                    mma_ts(d, tmem + C::kColQ + kk * 8, bd, C::kIdescQK, kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < C::kStepsR; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(qpe_addr + kk * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(sb + C::kChunksC * C::kChunk + kk * 32, 16, 1024);
-                    mma_ss(d, ad, bd, C::kIdescQK, 1u);
-                }
-                mma_commit(smem_addr(&bars.s_full[b]));
-                advance_unit(qpos, seq_lens, p.B, p.max_pages, p.gc);
-                return true;
-            };
-            // PV cursor
-            UnitPos vpos = pos0;
-            int vseg = -1;
-            bool vexact = false;
-            auto issue_pv = [&](long long t, bool first) -> bool {
-                const int b = (int)(t & 1);
-                if (!wt.wait(smem_addr(&bars.p_full[b]), (uint32_t)((t >> 1) & 1))) return false;
-                if (first && vseg > 0 && !wt.wait(smem_addr(&bars.o_free), (uint32_t)((vseg - 1) & 1))) return false;
-                tc_fence_after();
-                const uint32_t sb = stage0 + (int)(t % NST) * C::kStageBytes;
-                const uint32_t pa = p_addr + b * C::kPBytes;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(pa + kk * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(sb + kk * 2048, C::kChunk, 1024);
-                    mma_ss(tmem + C::kColO, ad, bd, vexact ? C::kIdescPVf16 : C::kIdescPVbf16,
-                           (first && kk == 0) ? 0u : 1u);
-                }
-                mma_commit(smem_addr(&bars.empty[(int)(t % NST)]));
-                mma_commit(smem_addr(&bars.o_done[b]));
-                return true;
-            };
             // Issue whichever MMA is ready, polling without blocking: QK^T of the next tile as
-            // soon as its stage has landed and its S buffer is free, PV of the oldest tile as
-            // soon as its P is in shared memory.  Neither stream waits on the other.
+            // soon as its stage has landed and S has been read, PV of the oldest tile as soon as
+            // its P is in shared memory.  Each stream has its own tile cursor.
+            Tile tq = make_tile(pos0, lo, lo, hi), tv = tq;
             long long jq = 0, jv = 0;
-            bool vbegun = false;
+            int qseg = -1, vseg = -1;
+            bool vbegun = false, vexact = false;
             long long idle_since = clock64();
-            while (ok && jv < n) {
+            while (ok && tv.u < hi) {
                 bool did = false;
-                if (jq < n) {
-                    const SegFlags fq = seg_flags(lo + jq, lo, hi, qpos);
-                    const int st = (int)(jq % NST), b = (int)(jq & 1);
-                    if ((!fq.begin || mbar_test_wait(smem_addr(&bars.q_full), (uint32_t)((qseg + 1) & 1))) &&
+                if (tq.u < hi) {
+                    const int st = (int)(jq % NST);
+                    if ((!tq.begin || mbar_test_wait(smem_addr(&bars.q_full), (uint32_t)((qseg + 1) & 1))) &&
                         mbar_test_wait(smem_addr(&bars.full[st]), (uint32_t)((jq / NST) & 1)) &&
-                        (jq < 2 || mbar_test_wait(smem_addr(&bars.s_free[b]), (uint32_t)(((jq >> 1) - 1) & 1)))) {
-                        ok = issue_qk(jq);       // its waits are already satisfied
+                        (jq == 0 || mbar_test_wait(smem_addr(&bars.s_free), (uint32_t)((jq - 1) & 1)))) {
+                        if (tq.begin) ++qseg;
+                        tc_fence_after();
+                        const uint32_t sb = stage0 + st * C::kStageBytes;
+                        const uint32_t d = tmem + C::kColS;
+#pragma unroll
+                        for (int kk = 0; kk < C::kStepsC; ++kk) {
+                            const uint64_t bd = smem_desc_sw128(sb + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024);
+                            mma_ts(d, tmem + C::kColQ + kk * 8, bd, C::kIdescQK, kk > 0 ? 1u : 0u);
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < C::kStepsR; ++kk) {
+                            const uint64_t ad = smem_desc_sw128(qpe_addr + kk * 32, 16, 1024);
+                            const uint64_t bd = smem_desc_sw128(sb + C::kChunksC * C::kChunk + kk * 32, 16, 1024);
+                            mma_ss(d, ad, bd, C::kIdescQK, 1u);
+                        }
+                        mma_commit(smem_addr(&bars.s_full));
+                        tq = next_tile(tq, seq_lens, p, lo, hi);
                         ++jq;
                         did = true;
                     }
                 }
-                if (ok && jv < jq) {
-                    const SegFlags fv = seg_flags(lo + jv, lo, hi, vpos);
-                    if (fv.begin && !vbegun) {
+                if (jv < jq) {
+                    if (tv.begin && !vbegun) {
                         ++vseg;
-                        vexact = vpos.T < kExactPVBelow;
+                        vexact = tv.pos.T < kExactPVBelow;
                         vbegun = true;
                     }
-                    const int b = (int)(jv & 1);
-                    if (mbar_test_wait(smem_addr(&bars.p_full[b]), (uint32_t)((jv >> 1) & 1)) &&
-                        (!fv.begin || vseg == 0 ||
+                    if (mbar_test_wait(smem_addr(&bars.p_full), (uint32_t)(jv & 1)) &&
+                        (!tv.begin || vseg == 0 ||
                          mbar_test_wait(smem_addr(&bars.o_free), (uint32_t)((vseg - 1) & 1)))) {
-                        ok = issue_pv(jv, fv.begin);
-                        advance_unit(vpos, seq_lens, p.B, p.max_pages, p.gc);
+                        tc_fence_after();
+                        const int st = (int)(jv % NST);
+                        const uint32_t sb = stage0 + st * C::kStageBytes;
+#pragma unroll
+                        for (int kk = 0; kk < kTileTok / 16; ++kk) {
+                            // A: 16 tokens of P (K-major); B: the same 16 token rows of every latent chunk (MN-major)
+                            const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * C::kPChunk + (kk & 3) * 32, 16, 1024);
+                            const uint64_t bd = smem_desc_sw128(sb + kk * 2048, C::kChunk, 1024);
+                            mma_ss(tmem + C::kColO, ad, bd, vexact ? C::kIdescPVf16 : C::kIdescPVbf16,
+                                   (tv.begin && kk == 0) ? 0u : 1u);
+                        }
+                        mma_commit(smem_addr(&bars.empty[st]));
+                        mma_commit(smem_addr(&bars.o_done));
+                        tv = next_tile(tv, seq_lens, p, lo, hi);
                         ++jv;
                         vbegun = false;
                         did = true;
@@ -391,28 +409,32 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         const bool warp_active = quad * 32 < p.H;
         const bool row_active = row < p.H;
         const int tid_sm = threadIdx.x - kSoftmaxWarp0 * 32;   // 0..255
-        const float sc = p.scale_log2;
+        // A negative scale is folded into the query: its bf16 sign bits are flipped on load (exact),
+        // so the scores this kernel sees are multiplied by |scale| and the row maximum is the max.
+        const float sc = fabsf(p.scale_log2);
+        const uint32_t qflip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
         constexpr int kOHalf = LS / 2;                    // O columns per warpgroup
-        UnitPos pos = pos0;
+        constexpr int kCols = kTileTok / 2;               // score columns per warpgroup
         long long last_o = -1;                            // highest PV index whose completion was observed
         int seg = -1;
         float m = -INFINITY, l = 0.f;                     // l: this warpgroup's half of the row sum
         bool first_tile = true;
         bool exact = false;                               // fp16 PV for this segment
-        // PV(t) completes on o_done[t & 1]; completions are in order, so observing PV(t) covers all before it
+        // PV(t) is the t-th completion of o_done; completions are in order, so observing PV(t)
+        // covers all before it
         auto wait_o = [&](long long t) -> bool {
             if (t <= last_o) return true;
-            if (!wt.wait(smem_addr(&bars.o_done[t & 1]), (uint32_t)((t >> 1) & 1))) return false;
+            if (!wt.wait(smem_addr(&bars.o_done), (uint32_t)(t & 1))) return false;
             last_o = t;
             tc_fence_after();
             return true;
         };
+        Tile t = make_tile(pos0, lo, lo, hi);
         long long j = 0;
-        for (; j < n; ++j) {
-            const SegFlags f = seg_flags(lo + j, lo, hi, pos);
+        for (; t.u < hi; ++j) {
+            const UnitPos pos = t.pos;
             const int shard = p.shard0 + pos.s;
-            const int buf = (int)(j & 1);
-            if (f.begin) {
+            if (t.begin) {
                 ++seg;
                 // query of this (b, shard): the latent part into tensor memory as bf16 pairs
                 // (warpgroups take alternate 64-element chunks), the RoPE part into shared memory
@@ -426,7 +448,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                         for (int v = 0; v < 8; ++v) {
                             uint4 x = make_uint4(0, 0, 0, 0);
                             if (row_active) x = __ldg(qs + c * 8 + v);
-                            r[4 * v + 0] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+                            r[4 * v + 0] = x.x ^ qflip; r[4 * v + 1] = x.y ^ qflip; r[4 * v + 2] = x.z ^ qflip; r[4 * v + 3] = x.w ^ qflip;
                         }
                         tmem_st32(lane_base + C::kColQ + c * 32, r);
                     }
@@ -438,7 +460,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                     for (int k = 0; k < 4; ++k) {
                         const int c = wg * 4 + k;
                         const uint4 x = row_active ? __ldg(qp + c) : make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4*>(qpe_smem + sw128_offset(row, c)) = x;
+                        *reinterpret_cast<uint4*>(qpe_smem + sw128_offset(row, c)) = make_uint4(x.x ^ qflip, x.y ^ qflip, x.z ^ qflip, x.w ^ qflip);
                     }
                     fence_proxy_async_smem();
                 }
@@ -450,48 +472,50 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 first_tile = true;
                 exact = pos.T < kExactPVBelow;
             }
-            const int valid = min(kPage, pos.T - pos.tile * kPage);
-            const bool tail = valid < kPage;
-            if (!wt.wait(smem_addr(&bars.s_full[buf]), (uint32_t)((j >> 1) & 1))) break;
+            // tokens of this tile that belong to the sequence (rows 0-63 the first page, 64-127 the second)
+            const int loaded = t.npages * kPage;
+            const int valid = min(loaded, pos.T - pos.tile * kPage);
+            const bool tail = valid < kTileTok;
+            if (!wt.wait(smem_addr(&bars.s_full), (uint32_t)(j & 1))) break;
             tc_fence_after();
-            uint32_t sraw[32];
-            if (warp_active) tmem_ld32(lane_base + C::kColS + buf * 64 + wg * 32, sraw);
-            uint8_t* sb = smem + (int)(j % NST) * C::kStageBytes;
-            if (warp_active) tmem_wait_ld();
-            tc_fence_before();
-            warp_arrive(smem_addr(&bars.s_free[buf]));
-
-            // row extreme of the raw scores over this warpgroup's 32 columns
-            // (the maximum of scale * s is scale * max(s) for scale >= 0, scale * min(s) otherwise)
-            float s[32];
-#pragma unroll
-            for (int t = 0; t < 32; ++t) s[t] = __uint_as_float(sraw[t]);
-            float ext = sc >= 0.f ? -INFINITY : INFINITY;
+            float s[kCols];
             if (warp_active) {
-                if (!tail) {
-                    float e4[4];
+                uint32_t r0[32], r1[32];
+                tmem_ld32(lane_base + C::kColS + wg * kCols, r0);
+                tmem_ld32(lane_base + C::kColS + wg * kCols + 32, r1);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) e4[k] = s[k];
-                    if (sc >= 0.f) {
-#pragma unroll
-                        for (int t = 4; t < 32; ++t) e4[t & 3] = fmaxf(e4[t & 3], s[t]);
-                        ext = fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]));
-                    } else {
-#pragma unroll
-                        for (int t = 4; t < 32; ++t) e4[t & 3] = fminf(e4[t & 3], s[t]);
-                        ext = fminf(fminf(e4[0], e4[1]), fminf(e4[2], e4[3]));
-                    }
-                } else {
-#pragma unroll
-                    for (int t = 0; t < 32; ++t)
-                        if (wg * 32 + t < valid) ext = sc >= 0.f ? fmaxf(ext, s[t]) : fminf(ext, s[t]);
+                for (int k = 0; k < 32; ++k) {
+                    s[k] = __uint_as_float(r0[k]);
+                    s[k + 32] = __uint_as_float(r1[k]);
                 }
+            } else {
+#pragma unroll
+                for (int k = 0; k < kCols; ++k) s[k] = 0.f;
+            }
+            tc_fence_before();
+            warp_arrive(smem_addr(&bars.s_free));
+            uint8_t* sb = smem + (int)(j % NST) * C::kStageBytes;
+
+            // row maximum of the raw scores over this warpgroup's valid columns
+            float ext = -INFINITY;
+            if (warp_active) {
+                if (tail) {
+#pragma unroll
+                    for (int k = 0; k < kCols; ++k) s[k] = wg * kCols + k < valid ? s[k] : -INFINITY;
+                }
+                float e4[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) e4[k] = s[k];
+#pragma unroll
+                for (int k = 4; k < kCols; ++k) e4[k & 3] = fmaxf(e4[k & 3], s[k]);
+                ext = fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]));
             }
             bars.xmax_buf[j & 1][wg][row] = ext;
             warp_arrive(smem_addr(&bars.xmax));
             if (!wt.wait(smem_addr(&bars.xmax), (uint32_t)(j & 1))) break;
             const float other = bars.xmax_buf[j & 1][wg ^ 1][row];
-            const float mt = (sc >= 0.f ? fmaxf(ext, other) : fminf(ext, other)) * sc;   // max of scale*s
+            const float mt = fmaxf(ext, other) * sc;   // max of scale*s
 
             bool alive = true;
             if (warp_active) {
@@ -522,40 +546,41 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 }
             }
             if (!alive) break;
-            uint32_t pk[16];
+            uint32_t pk[kCols / 2];
             if (warp_active) {
                 const float nm = -m;
                 // even columns on the special-function unit, odd columns on the FMA pipe
 #pragma unroll
-                for (int t = 0; t < 32; ++t)
-                    s[t] = (t & 1) ? ex2_fma(fmaf(s[t], sc, nm)) : ex2_approx(fmaf(s[t], sc, nm));
+                for (int k = 0; k < kCols; ++k)
+                    s[k] = ex2_approx(fmaf(s[k], sc, nm));
                 if (tail) {
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) s[t] = wg * 32 + t < valid ? s[t] : 0.f;
+                    for (int k = 0; k < kCols; ++k) s[k] = wg * kCols + k < valid ? s[k] : 0.f;
                 }
                 float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int t = 0; t < 32; ++t) l4[t & 3] += s[t];
+                for (int k = 0; k < kCols; ++k) l4[k & 3] += s[k];
                 l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
                 if (exact) {
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) pk[t] = pack_f16x2(s[2 * t], s[2 * t + 1]);
+                    for (int k = 0; k < kCols / 2; ++k) pk[k] = pack_f16x2(s[2 * k], s[2 * k + 1]);
                 } else {
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(s[2 * t], s[2 * t + 1]);
+                    for (int k = 0; k < kCols / 2; ++k) pk[k] = pack_bf16x2(s[2 * k], s[2 * k + 1]);
                 }
             } else {
 #pragma unroll
-                for (int t = 0; t < 16; ++t) pk[t] = 0u;
+                for (int k = 0; k < kCols / 2; ++k) pk[k] = 0u;
             }
             if (exact) {
                 // this tile's latent rows -> fp16 (rows past the sequence end -> 0) for PV;
-                // QK^T has finished reading them
-#pragma unroll
+                // QK^T has finished reading them.  The 128B swizzle only permutes the 16-byte
+                // pieces within a row, so row rr is the 128 bytes at rr * 128 of its chunk.
+#pragma unroll 4
                 for (int k = 0; k < C::kCvt; ++k) {
                     const int i = tid_sm + k * kSoftmaxWarps * 32;
-                    const int rr = (i >> 3) & 63;
-                    uint4* ptr = reinterpret_cast<uint4*>(sb + (i >> 9) * C::kChunk + rr * 128 + (i & 7) * 16);
+                    const int rr = (i >> 3) & (kTileTok - 1);
+                    uint4* ptr = reinterpret_cast<uint4*>(sb + (i >> 10) * C::kChunk + rr * 128 + (i & 7) * 16);
                     uint4 v = *ptr;
                     if (rr < valid) {
                         v.x = bf16x2_to_f16x2(v.x);
@@ -567,36 +592,37 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                     }
                     *ptr = v;
                 }
-            } else if (tail) {
-                // bf16 tile kept as it is; only the rows past the sequence end are zeroed
-                const int rows = kPage - valid;
+            } else if (valid < loaded) {
+                // bf16 tile kept as it is; only the loaded rows past the sequence end are zeroed
+                // (the rows of a page that was not loaded are zero already)
+                const int rows = loaded - valid;
                 for (int i = tid_sm; i < C::kChunksC * rows * 8; i += kSoftmaxWarps * 32) {
                     const int c = i / (rows * 8), rr = valid + (i / 8) % rows, seg16 = i % 8;
                     *reinterpret_cast<uint4*>(sb + c * C::kChunk + rr * 128 + seg16 * 16) = make_uint4(0, 0, 0, 0);
                 }
             }
-            // P buffer `buf` is free once PV(j - 2), its last reader, has completed
-            if (j >= 2 && !wait_o(j - 2)) break;
+            // the P buffer is free once PV(j - 1), its last reader, has completed
+            if (j >= 1 && !wait_o(j - 1)) break;
             {
-                uint8_t* pb = p_smem + buf * C::kPBytes;
+                uint8_t* pb = p_smem + wg * C::kPChunk;   // this warpgroup's 64 tokens: one K chunk of P
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    *reinterpret_cast<uint4*>(pb + sw128_offset(row, wg * 4 + k)) =
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<uint4*>(pb + sw128_offset(row, k)) =
                         make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
             }
             fence_proxy_async_smem();
-            warp_arrive(smem_addr(&bars.p_full[buf]));
+            warp_arrive(smem_addr(&bars.p_full));
             first_tile = false;
 
-            if (f.end) {
+            if (t.end) {
                 if (!wait_o(j)) break;
                 // the two warpgroups' halves of the softmax sum
                 bars.xsum_buf[seg & 1][wg][row] = l;
                 warp_arrive(smem_addr(&bars.xsum));
                 if (!wt.wait(smem_addr(&bars.xsum), (uint32_t)(seg & 1))) break;
                 const float lt = l + bars.xsum_buf[seg & 1][wg ^ 1][row];
-                const long long u = lo + j;
-                const long long seg_first = (u - pos.tile) < lo ? lo : (u - pos.tile);
+                const long long u_first = t.u - pos.tile;       // unit of page 0 of this (b, s)
+                const long long seg_first = u_first < lo ? lo : u_first;
                 const int slot = seg_first == lo ? w : p.W + pos.b * p.gc + pos.s;
                 if (warp_active) {
                     const float inv_l = 1.0f / lt;
@@ -620,7 +646,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 tc_fence_before();
                 warp_arrive(smem_addr(&bars.o_free));
             }
-            advance_unit(pos, seq_lens, p.B, p.max_pages, p.gc);
+            t = next_tile(t, seq_lens, p, lo, hi);
         }
     }
 
@@ -695,9 +721,9 @@ cudaError_t launch_attention_sm100(const Plan& p, const __nv_bfloat16* q, const 
                                    int wait_limit_us, int debug_stall, cudaStream_t stream) {
     const uint64_t wait_ns = (wait_limit_us > 0 ? (uint64_t)wait_limit_us : 1000000ull) * 1000ull;
     switch (p.Ls) {
-        case 256: return launch_t<256, 64, 4>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
-        case 128: return launch_t<128, 64, 6>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
-        case 64: return launch_t<64, 64, 10>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
+        case 256: return launch_t<256, 64, 2>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
+        case 128: return launch_t<128, 64, 3>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
+        case 64: return launch_t<64, 64, 5>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
     }
     return cudaErrorNotSupported;
 }

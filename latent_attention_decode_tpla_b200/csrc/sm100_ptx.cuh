@@ -74,12 +74,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint
         : "memory");
 }
 
-// bring a tile into L2 only (no shared memory, no barrier)
-__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(x), "r"(y)
-                 : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -159,39 +153,11 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-
 // 2^x on the special-function unit (PTX ex2.approx, subnormal results flushed to zero)
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// 2^x on the FMA and integer pipes, for x <= 0 (the special-function unit is the
-// softmax's bottleneck, so part of the exponentials are computed here instead).
-// Range reduction x = i + f with i = round(x) (adding 1.5 * 2^23 rounds x to an
-// integer held in the low mantissa bits) and f in [-0.5, 0.5]; 2^f by a
-// degree-4 polynomial fitted to 2^f on that interval for least maximum relative
-// error (2.7e-6, well under the 16-bit rounding of P that follows); 2^i is added
-// to the exponent field.  Inputs below -120 are clamped (2^-120 is zero at the
-// precision that matters here).
-__device__ __forceinline__ float ex2_fma(float x) {
-    x = fmaxf(x, -120.0f);
-    const float t = x + 12582912.0f;
-    const float f = x - (t - 12582912.0f);
-    float y = fmaf(0.009570068679749966f, f, 0.055917806923389435f);
-    y = fmaf(y, f, 0.240247443318367f);
-    y = fmaf(y, f, 0.6931218504905701f);
-    y = fmaf(y, f, 0.9999992847442627f);
-    return __int_as_float(__float_as_int(y) + (__float_as_int(t) << 23));
 }
 
 // ------------------------------------------------------------------ descriptors

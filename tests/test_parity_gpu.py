@@ -201,3 +201,16 @@ def test_pv_precision_modes_at_the_length_boundary(kernel):
     hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "all shards")
     hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=1, kernel=kernel),
                     hx.run_oracle(d, scale, mode="shard", shard=1), "shard 1")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("scale", [-1 / math.sqrt(192), 0.0, 0.5])
+def test_softmax_scale_sign_and_size(kernel, scale):
+    """A negative scale (the kernel folds its sign into the query), a zero scale (uniform
+    weights over the valid tokens, ragged tails included) and a large one (the row maximum
+    grows by more than the lazy-rescale threshold across tiles)."""
+    d = _case(4, 128, 512, 64, 128, 2, [300, 1, 129, 1000], seed=23)
+    _kernel_or_skip(d, kernel)
+    hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "scale %g" % scale)
+    hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=0, with_wuv=False, kernel=kernel),
+                    hx.run_oracle(d, scale, mode="shard", shard=0, with_wuv=False), "scale %g shard latent" % scale)
