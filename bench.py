@@ -467,8 +467,9 @@ def main():
                      "frac": achieved / peak, "traffic": profiled_traffic(kernel_name, spec["name"]),
                      "kernel": kernel_name + " (tpla_attention)", "peak_kind": peak_kind,
                      "bytes_per_launch": r["attn_bytes"], "us_per_launch": r["attn_ms"] * 1e3},
-        "e2e": {"value": r["total_cache"] / (r["e2e_ms"] * 1e-3) / 1e9, "unit": "GB/s",
-                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"]},
+        "e2e": None if args.no_e2e else {
+            "value": r["total_cache"] / (r["e2e_ms"] * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"]},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
