@@ -167,9 +167,8 @@ int mla_decode(const tpla_dims_t* dims,
  * loads the library holds until the process exits; the call allocates and
  * frees nothing (no cudaMalloc, no allocating library routine).
  *   - Size limit: the split-KV partials of B*g (sequence, shard) pairs plus at
- *     least one worker, and the merged outputs, must fit in 32 MiB, i.e.
- *     roughly (B*g + 1) * H * (L/g) * 4 + B * H * L * 4 bytes plus a small
- *     header; larger problems
+ *     least one worker must fit in 32 MiB, i.e. roughly
+ *     (B*g + 1) * H * (L/g) * 4 bytes plus a small header; larger problems
  *     return TPLA_ERR_WORKSPACE with nothing enqueued.  Near the limit the
  *     call uses fewer split-KV workers than tpla_decode (same result up to
  *     fp32 rounding, possibly slower).

@@ -56,19 +56,15 @@ size_t ws_lse_bytes(const tpla_dims_t* d) {
     return align_up((size_t)(kMaxWorkers + (size_t)d->B * d->g) * d->H * sizeof(float), 256);
 }
 
-// Workspace: 256-byte header | log-sum-exps [kMaxWorkers + B*g][H] | partial outputs [slots][H][L/g]
-// | merged shard outputs [B][H][L].  `slots` is kMaxWorkers + B*g for a caller's workspace.
+// Workspace: 256-byte header | log-sum-exps [kMaxWorkers + B*g][H] | partial outputs [slots][H][L/g].
+// `slots` is kMaxWorkers + B*g for a caller's workspace.
 size_t ws_part_bytes(const tpla_dims_t* d, size_t slots) {
     return align_up(slots * d->H * (size_t)(d->L / d->g) * sizeof(float), 256);
 }
 
-size_t ws_merged_bytes(const tpla_dims_t* d) {
-    return align_up((size_t)d->B * d->H * d->L * sizeof(float), 256);
-}
-
 size_t ws_bytes_for(const tpla_dims_t* d) {
     const size_t slots = (size_t)kMaxWorkers + (size_t)d->B * d->g;
-    return 256 + ws_lse_bytes(d) + ws_part_bytes(d, slots) + ws_merged_bytes(d);
+    return 256 + ws_lse_bytes(d) + ws_part_bytes(d, slots);
 }
 
 int device_info(unsigned** status, int* sms) {
@@ -134,7 +130,6 @@ Workspace carve(void* workspace, const tpla_dims_t* d, size_t slots = 0) {
     Workspace w;
     w.part_lse = reinterpret_cast<float*>(base);
     w.part_o = reinterpret_cast<float*>(base + ws_lse_bytes(d));
-    w.merged = reinterpret_cast<float*>(base + ws_lse_bytes(d) + ws_part_bytes(d, slots));
     return w;
 }
 
@@ -384,8 +379,8 @@ extern "C" int tpla_decode_static(const tpla_dims_t* dims, const tpla_bf16* q, c
     if (block_table && !aligned16(block_table)) return TPLA_ERR_INVALID_ARG;
     if (w_uv && !aligned16(w_uv)) return TPLA_ERR_INVALID_ARG;
     if (!block_table && (long long)dims->B * dims->max_pages_per_seq > dims->num_pages) return TPLA_ERR_INVALID_ARG;
-    // partial slots that fit next to the header, the log-sum-exp block and the merged outputs
-    const size_t head = 256 + ws_lse_bytes(dims) + ws_merged_bytes(dims) + 256;
+    // partial slots that fit next to the header and the log-sum-exp block
+    const size_t head = 256 + ws_lse_bytes(dims) + 256;
     if (head >= kStaticScratchBytes) return TPLA_ERR_WORKSPACE;
     const size_t slot_bytes = (size_t)dims->H * (size_t)(dims->L / dims->g) * sizeof(float);
     const long long max_slots = (long long)((kStaticScratchBytes - head) / slot_bytes);

@@ -51,7 +51,12 @@ attn_simt_kernel(Plan p, const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     const long long U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
     if (U == 0) return;
     const long long lo = unit_lo(w, U, p.W), hi = unit_lo(w + 1, U, p.W);
-    if (lo >= hi) return;
+    if (lo >= hi) {
+        // a worker with no units leaves a zero-weight partial in its slot: the merge may count it
+        // as a segment of the pair it falls inside
+        for (int i = threadIdx.x; i < kHG && h0 + i < p.H; i += blockDim.x) ws.part_lse[(size_t)w * p.H + h0 + i] = -INFINITY;
+        return;
+    }
     UnitPos pos = warp_locate_unit(seq_lens, p.B, p.max_pages, p.gc, lo);
 
     float acc[NACC];

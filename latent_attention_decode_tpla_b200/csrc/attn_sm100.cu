@@ -207,7 +207,12 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     const long long U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
     if (U == 0) return;
     const long long lo = unit_lo(w, U, p.W), hi = unit_lo(w + 1, U, p.W);
-    if (lo >= hi) return;
+    if (lo >= hi) {
+        // a worker with no units leaves a zero-weight partial in its slot: the merge may count it
+        // as a segment of the pair it falls inside
+        for (int i = threadIdx.x; i < p.H; i += blockDim.x) ws.part_lse[(size_t)w * p.H + i] = -INFINITY;
+        return;
+    }
     const UnitPos pos0 = warp_locate_unit(seq_lens, p.B, p.max_pages, p.gc, lo);
 
     if (threadIdx.x == 0) {

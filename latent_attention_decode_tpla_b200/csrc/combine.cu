@@ -1,4 +1,4 @@
-// Combine: split-KV merge, W_UV up-projection, and the sum over shards.
+// Combine: split-KV merge, W_UV up-projection, and the sum over shards, in one kernel.
 //
 // For sequence b, head h and shard s the attention kernels left one partial
 // (o_k, lse_k) per split-KV segment k (o_k normalised by its own softmax
@@ -10,160 +10,229 @@
 //     out_{b,h} = sum_s W_UV_h[s*Ls:(s+1)*Ls, :]^T o_{b,h,s}      (fp32)
 // or, without W_UV, the shard outputs side by side.
 //
-// Two kernels, each a few dependent memory round trips deep:
-//   merge_kernel    one CTA per (sequence, shard, 8 heads): the segment list
-//                   of the (sequence, shard) is built once, then each warp
-//                   merges one head with independent vector loads and writes
-//                   o_{b,h,s} to the `merged` buffer (or straight to `out`
-//                   when there is no W_UV);
-//   project_kernel  one CTA per head (and dv slice): W_UV_h rows are copied
-//                   asynchronously into shared memory and reused for every
-//                   sequence of the batch.
+// One CTA per (head h, dv slice, group of Bc sequences):
+//   1. one thread starts the bulk copy of the CTA's W_UV rows into shared
+//      memory (a single copy when the slice is the whole dv);
+//   2. one warp finds, for each (sequence, shard) pair of the group, the
+//      workers holding its first and last tile (a prefix sum over seq_lens);
+//   3. every thread merges one 4-float piece of one pair's row over that
+//      pair's segments in a single pass (running maximum and rescale), so all
+//      partial and log-sum-exp loads are independent;
+//   4. the projection keeps kRows rows x 8 columns per lane in registers (one
+//      16-byte W_UV load per row of the reduction for 64 FMAs), sums the lanes'
+//      parts by shuffles and the warps' parts through shared memory.
+// The partials were just written by the attention kernel and come from L2.
 #include "tpla_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace tpla {
 namespace {
 
-constexpr int kMergeWarps = 8;                 // heads per merge CTA
-constexpr int kProjThreads = 256;
-constexpr int kProjChunk = 8;                  // sequences projected together (accumulators per thread)
-constexpr size_t kWSmemBudget = 128 * 1024;    // bytes of W_UV staged per projection CTA
+using namespace sm100;
 
-// Sum over sequences [b_begin, b_end) of gc * tiles, by one full warp.
-__device__ inline long long warp_units_range(const int32_t* seq_lens, int b_begin, int b_end, int max_pages, int gc) {
-    const int lane = threadIdx.x & 31;
-    long long acc = 0;
-    for (int base = b_begin; base < b_end; base += 32) {
-        const int b = base + lane;
-        if (b < b_end) {
-            int T = __ldg(seq_lens + b);
-            T = T < 0 ? 0 : (T > max_pages * kPage ? max_pages * kPage : T);
-            acc += tiles_of_len(T);
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr size_t kWSmemBudget = 64 * 1024;     // bytes of W_UV staged per CTA
+constexpr int kMergeTarget = 2048;             // merged floats per CTA the group size aims at
+constexpr int kRows = 8;                       // merged rows projected together
+constexpr int kMaxPairs = 64;                  // (sequence, shard) pairs per CTA
+
+// The schedule's unit boundaries lo(w) = floor(w U / W) and owners, in 32-bit arithmetic when
+// (W + 1) U fits (64-bit integer division is emulated and slow), else in 64 bits.
+struct UnitMath {
+    long long U;
+    int W;
+    bool small;
+    __device__ long long lo(long long w) const {
+        return small ? (long long)(((unsigned)w * (unsigned)U) / (unsigned)W) : unit_lo(w, U, W);
+    }
+    __device__ int worker(long long u) const {
+        return small ? (int)(((unsigned)(u + 1) * (unsigned)W - 1u) / (unsigned)U) : unit_worker(u, U, W);
+    }
+};
+
+struct PairInfo {
+    int wf, wl;        // workers holding the pair's first and last tile (wl < wf: empty sequence)
+    int first_slot;    // slot of the first segment
+};
+
+__global__ void __launch_bounds__(kThreads)
+combine_kernel(Plan p, int Bc, int dsub, const int32_t* __restrict__ seq_lens, Workspace ws,
+               const __nv_bfloat16* __restrict__ w_uv, float* __restrict__ out, uint64_t wait_cycles) {
+    extern __shared__ __align__(128) uint8_t csm[];
+    __shared__ PairInfo pinfo[kMaxPairs];
+    __shared__ __align__(8) uint64_t wbar;
+    const int Lc = p.gc * p.Ls;
+    const int h = blockIdx.x, d0 = blockIdx.y * dsub, b0 = blockIdx.z * Bc;
+    const int nb = min(Bc, p.B - b0);
+    const int npairs = nb * p.gc;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool project = w_uv != nullptr;
+    // shared memory: W_UV rows [Lc][dsub] bf16 | merged rows [Bc][Lc] fp32 | warps' partial sums
+    // [kWarps][kRows][dsub] fp32
+    __nv_bfloat16* w_s = reinterpret_cast<__nv_bfloat16*>(csm);
+    const size_t w_bytes = project ? (size_t)Lc * dsub * 2 : 0;
+    float* o_s = reinterpret_cast<float*>(csm + w_bytes);
+    float* red = o_s + (size_t)Bc * Lc;
+
+    // 1. W_UV[h][shard0*Ls + j][d0 .. d0+dsub) for j < Lc
+    if (project && warp == 0) {
+        if (lane == 0) {
+            mbar_init(smem_addr(&wbar), 1);
+            fence_barrier_init();
+            mbar_arrive_expect_tx(smem_addr(&wbar), (uint32_t)w_bytes);
+        }
+        __syncwarp();
+        const __nv_bfloat16* src = w_uv + ((size_t)h * p.L + (size_t)p.shard0 * p.Ls) * p.dv + d0;
+        if (dsub == p.dv) {
+            if (lane == 0) bulk_load(smem_addr(w_s), src, (uint32_t)w_bytes, smem_addr(&wbar));
+        } else {
+            for (int j = lane; j < Lc; j += 32)
+                bulk_load(smem_addr(w_s + (size_t)j * dsub), src + (size_t)j * p.dv, (uint32_t)(dsub * 2),
+                          smem_addr(&wbar));
         }
     }
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    return acc * gc;
-}
-
-__global__ void __launch_bounds__(kMergeWarps * 32)
-merge_kernel(Plan p, const int32_t* __restrict__ seq_lens, Workspace ws, float* __restrict__ dst_base,
-             int dst_cols) {
-    __shared__ int s_slot[kMaxWorkers + 1];
-    __shared__ int s_nseg;
-    const int b = blockIdx.y / p.gc, s = blockIdx.y % p.gc;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.x * kMergeWarps + warp;
-
-    int T = __ldg(seq_lens + b);
-    T = T < 0 ? 0 : (T > p.max_pages * kPage ? p.max_pages * kPage : T);
-    const int nt = tiles_of_len(T);
-    if (warp == 0 && nt > 0) {
-        // segments of (b, s): the worker holding its first tile, then every later
-        // non-empty worker up to the one holding its last tile
-        const long long U = warp_units_range(seq_lens, 0, p.B, p.max_pages, p.gc);
-        const long long u0 = warp_units_range(seq_lens, 0, b, p.max_pages, p.gc) + (long long)s * nt;
-        const long long u1 = u0 + nt - 1;
-        const int wf = unit_worker(u0, U, p.W), wl = unit_worker(u1, U, p.W);
-        if (lane == 0) s_slot[0] = unit_lo(wf, U, p.W) == u0 ? wf : p.W + b * p.gc + s;
-        int n = 1;
-        for (int base = wf + 1; base <= wl; base += 32) {
-            const int wk = base + lane;
-            const bool ok = wk <= wl && unit_lo(wk, U, p.W) < unit_lo(wk + 1, U, p.W);
-            const unsigned m = __ballot_sync(0xffffffffu, ok);
-            if (ok) s_slot[n + __popc(m & ((1u << lane) - 1u))] = wk;
-            n += __popc(m);
+    // 2. first and last worker of each pair: prefix sum of tiles over the sequences before b
+    if (warp == (project ? 1 : 0)) {
+        UnitMath um;
+        um.U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
+        um.W = p.W;
+        um.small = um.U < (1ll << 32) / (p.W + 1);
+        long long before = 0;                         // units of sequences < base
+        for (int base = 0; base < b0 + nb; base += 32) {
+            const int b = base + lane;
+            int nt = 0;
+            if (b < b0 + nb) {
+                int T = __ldg(seq_lens + b);
+                T = T < 0 ? 0 : (T > p.max_pages * kPage ? p.max_pages * kPage : T);
+                nt = tiles_of_len(T);
+            }
+            long long incl = (long long)nt * p.gc;   // inclusive scan over the lanes
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (b >= b0 && b < b0 + nb) {
+                const long long ub = before + incl - (long long)nt * p.gc;   // first unit of sequence b
+                for (int s = 0; s < p.gc; ++s) {
+                    PairInfo pi;
+                    if (nt == 0) {
+                        pi.wf = 0; pi.wl = -1; pi.first_slot = 0;
+                    } else {
+                        const long long u0 = ub + (long long)s * nt;
+                        pi.wf = um.worker(u0);
+                        pi.wl = um.worker(u0 + nt - 1);
+                        pi.first_slot = um.lo(pi.wf) == u0 ? pi.wf : p.W + b * p.gc + s;
+                    }
+                    pinfo[(b - b0) * p.gc + s] = pi;
+                }
+            }
+            before += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) s_nseg = n;
     }
     __syncthreads();
-    if (h >= p.H) return;
-    float* dst = dst_base + ((size_t)b * p.H + h) * dst_cols + (size_t)s * p.Ls;
-    if (nt == 0) {
-        for (int j = lane * 4; j < p.Ls; j += 128) *reinterpret_cast<float4*>(dst + j) = make_float4(0, 0, 0, 0);
-        return;
-    }
-    const int n = s_nseg;
-    // softmax weights of the segments for this head
-    float M = -INFINITY;
-    for (int k = lane; k < n; k += 32) M = fmaxf(M, __ldg(ws.part_lse + (size_t)s_slot[k] * p.H + h));
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float den = 0.f;
-    for (int k = lane; k < n; k += 32) den += exp2f(__ldg(ws.part_lse + (size_t)s_slot[k] * p.H + h) - M);
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    const float inv = 1.0f / den;
-    for (int j = lane * 4; j < p.Ls; j += 128) {
-        float4 acc = make_float4(0, 0, 0, 0);
+
+    // 3. merge: one float4 of one pair's row per thread and iteration
+    const int q4 = p.Ls / 4;
+    for (int i = tid; i < npairs * q4; i += kThreads) {
+        const int pr = i / q4, j = (i % q4) * 4;
+        const int bl = pr / p.gc, s = pr % p.gc;
+        const PairInfo pi = pinfo[pr];
+        float M = -INFINITY, den = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        // segments: the first one, then one per later worker up to the last.  A worker with an
+        // empty range (possible when there are fewer units than workers) left lse = -inf in its
+        // slot, so its weight is 0 and its partial, never written, is not read into the sum.  No
+        // load depends on another, so they are all in flight together.
 #pragma unroll 8
-        for (int k = 0; k < n; ++k) {
-            const size_t slot = (size_t)s_slot[k];
-            const float wk = exp2f(__ldg(ws.part_lse + slot * p.H + h) - M) * inv;
-            const float4 v = __ldg(reinterpret_cast<const float4*>(ws.part_o + (slot * p.H + h) * p.Ls + j));
-            acc.x = fmaf(wk, v.x, acc.x);
-            acc.y = fmaf(wk, v.y, acc.y);
-            acc.z = fmaf(wk, v.z, acc.z);
-            acc.w = fmaf(wk, v.w, acc.w);
+        for (int k = pi.wf; k <= pi.wl; ++k) {
+            const size_t slot = (size_t)(k == pi.wf ? pi.first_slot : k);
+            const float lse = __ldg(ws.part_lse + slot * p.H + h);
+            float4 v = __ldg(reinterpret_cast<const float4*>(ws.part_o + (slot * p.H + h) * p.Ls + j));
+            const float Mn = fmaxf(M, lse);
+            const float a = exp2f(M - Mn), wk = exp2f(lse - Mn);   // exp2f(-inf) = 0 on the first segment
+            if (wk == 0.f) v = make_float4(0.f, 0.f, 0.f, 0.f);
+            den = den * a + wk;
+            acc.x = acc.x * a + wk * v.x;
+            acc.y = acc.y * a + wk * v.y;
+            acc.z = acc.z * a + wk * v.z;
+            acc.w = acc.w * a + wk * v.w;
+            M = Mn;
         }
-        *reinterpret_cast<float4*>(dst + j) = acc;
+        const float inv = pi.wl >= pi.wf ? 1.0f / den : 0.f;
+        const float4 r = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        if (project) {
+            *reinterpret_cast<float4*>(o_s + (size_t)bl * Lc + s * p.Ls + j) = r;
+        } else {
+            *reinterpret_cast<float4*>(out + ((size_t)(b0 + bl) * p.H + h) * Lc + s * p.Ls + j) = r;
+        }
     }
-}
-
-__global__ void __launch_bounds__(kProjThreads)
-project_kernel(Plan p, int dsub, const __nv_bfloat16* __restrict__ w_uv, const float* __restrict__ merged,
-               float* __restrict__ out) {
-    extern __shared__ __align__(16) uint8_t psm[];
-    const int Lc = p.gc * p.Ls;
-    __nv_bfloat16* w_s = reinterpret_cast<__nv_bfloat16*>(psm);                    // [Lc][dsub]
-    float* o_s = reinterpret_cast<float*>(psm + (size_t)Lc * dsub * 2);            // [chunk][Lc]
-    float* red = o_s + kProjChunk * Lc;                                             // [groups][chunk][dsub]
-    const int h = blockIdx.x;
-    const int d0 = blockIdx.y * dsub;
-    const int tid = threadIdx.x;
-
-    {   // W_UV[h][row0 + j][d0 .. d0+dsub) for j < Lc, 16-byte asynchronous copies
-        const size_t row0 = (size_t)p.shard0 * p.Ls;
-        const int per_row = dsub / 8;
-        const int n = Lc * per_row;
-        const uint4* src = reinterpret_cast<const uint4*>(w_uv);
-        for (int i = tid; i < n; i += kProjThreads) {
-            const int j = i / per_row, c = i % per_row;
-            const uint4* g = src + (((size_t)h * p.L + row0 + j) * p.dv + d0) / 8 + c;
-            const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(reinterpret_cast<uint4*>(w_s) + i));
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(g) : "memory");
+    if (!project) return;
+    for (int i = nb * Lc + tid; i < Bc * Lc; i += kThreads) o_s[i] = 0.f;   // rows past the batch
+    {   // wait for W_UV (bounded; a time-out is recorded in the device status)
+        const long long t0 = clock64();
+        while (!mbar_try_wait(smem_addr(&wbar), 0)) {
+            if ((uint64_t)(clock64() - t0) > wait_cycles) {
+                if (tid == 0) atomicOr(p.status, kStatusTimeout);
+                break;
+            }
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    const int groups = kProjThreads / dsub;
-    const int d = tid % dsub, grp = tid / dsub;
-    for (int c0 = 0; c0 < p.B; c0 += kProjChunk) {
-        const int nb = min(kProjChunk, p.B - c0);
-        // merged rows of this head for the chunk of sequences (rows past nb are zero)
-        for (int i = tid; i < kProjChunk * Lc / 4; i += kProjThreads) {
-            const int bl = i / (Lc / 4), j4 = i % (Lc / 4);
-            reinterpret_cast<float4*>(o_s)[i] =
-                bl < nb ? __ldg(reinterpret_cast<const float4*>(merged + ((size_t)(c0 + bl) * p.H + h) * Lc) + j4)
-                        : make_float4(0, 0, 0, 0);
-        }
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncthreads();
-        if (grp < groups) {
-            float acc[kProjChunk];
+    __syncthreads();
+
+    // 4. projection: out[b][d0 + 8c + e] = sum_j o[b][j] * W[j][8c + e].  Lane = (column group c of 8,
+    // part of this warp's slice of j).
+    const int cg = dsub / 8, ppw = 32 / cg;
+    const int cgi = lane % cg, part = lane / cg;
+    const int nparts = kWarps * ppw;
+    const int jpp = (Lc + nparts - 1) / nparts;
+    const int j0 = min(Lc, (warp * ppw + part) * jpp), j1 = min(Lc, j0 + jpp);
+    for (int r0 = 0; r0 < nb; r0 += kRows) {
+        float acc[kRows][8];
 #pragma unroll
-            for (int bl = 0; bl < kProjChunk; ++bl) acc[bl] = 0.f;
-#pragma unroll 4
-            for (int j = grp; j < Lc; j += groups) {
-                const float wv = __bfloat162float(w_s[(size_t)j * dsub + d]);
+        for (int r = 0; r < kRows; ++r)
 #pragma unroll
-                for (int bl = 0; bl < kProjChunk; ++bl) acc[bl] = fmaf(o_s[bl * Lc + j], wv, acc[bl]);
+            for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
+        const float* orow = o_s + (size_t)r0 * Lc;
+#pragma unroll 2
+        for (int j = j0; j < j1; ++j) {
+            const uint4 wv = *reinterpret_cast<const uint4*>(w_s + (size_t)j * dsub + cgi * 8);
+            const uint32_t wwords[4] = {wv.x, wv.y, wv.z, wv.w};
+            float wf[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                wf[2 * e] = __uint_as_float(wwords[e] << 16);
+                wf[2 * e + 1] = __uint_as_float(wwords[e] & 0xFFFF0000u);
             }
 #pragma unroll
-            for (int bl = 0; bl < kProjChunk; ++bl) red[(grp * kProjChunk + bl) * dsub + d] = acc[bl];
+            for (int r = 0; r < kRows; ++r) {
+                const float ov = orow[(size_t)r * Lc + j];   // rows past nb are zero
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(ov, wf[e], acc[r][e]);
+            }
+        }
+        for (int off = cg; off < 32; off <<= 1)
+#pragma unroll
+            for (int r = 0; r < kRows; ++r)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[r][e] += __shfl_xor_sync(0xffffffffu, acc[r][e], off);
+        if (part == 0) {
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+                float4* dst = reinterpret_cast<float4*>(red + ((size_t)warp * kRows + r) * dsub + cgi * 8);
+                dst[0] = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+                dst[1] = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
+            }
         }
         __syncthreads();
-        for (int i = tid; i < nb * dsub; i += kProjThreads) {
-            const int bl = i / dsub, dd = i % dsub;
-            float sum = 0.f;
-            for (int gi = 0; gi < groups; ++gi) sum += red[(gi * kProjChunk + bl) * dsub + dd];
-            out[((size_t)(c0 + bl) * p.H + h) * p.dv + d0 + dd] = sum;
+        for (int i = tid; i < kRows * dsub; i += kThreads) {
+            const int r = i / dsub, dd = i % dsub;
+            if (r0 + r < nb) {
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) sum += red[((size_t)w * kRows + r) * dsub + dd];
+                out[((size_t)(b0 + r0 + r) * p.H + h) * p.dv + d0 + dd] = sum;
+            }
         }
         __syncthreads();
     }
@@ -175,26 +244,29 @@ cudaError_t launch_combine(const Plan& p, const int32_t* seq_lens, const __nv_bf
                            float* out, Workspace ws, cudaStream_t stream) {
     if (p.B == 0) return cudaSuccess;
     const int Lc = p.gc * p.Ls;
-    dim3 mgrid((p.H + kMergeWarps - 1) / kMergeWarps, p.B * p.gc);
-    if (w_uv == nullptr) {
-        merge_kernel<<<mgrid, kMergeWarps * 32, 0, stream>>>(p, seq_lens, ws, out, Lc);
-        return cudaGetLastError();
+    // sequences per CTA: about kMergeTarget merged floats per CTA, whole row chunks when projecting
+    int Bc = kMergeTarget / Lc;
+    Bc = Bc < 1 ? 1 : (Bc > p.B ? p.B : Bc);
+    if (w_uv) Bc = (Bc + kRows - 1) / kRows * kRows;
+    while (Bc * p.gc > kMaxPairs) Bc = Bc > kRows ? Bc - kRows : Bc / 2;
+    if (Bc < 1) return cudaErrorNotSupported;
+    // dv slice: the widest 8 * 2^k columns (at most 256) that divide dv and whose W_UV rows fit the
+    // shared-memory budget (dv % 8 == 0)
+    int dsub = 8;
+    if (w_uv) {
+        while (dsub * 2 <= 256 && p.dv % (dsub * 2) == 0 && (size_t)Lc * dsub * 4 <= kWSmemBudget) dsub *= 2;
+        if ((size_t)Lc * dsub * 2 > kWSmemBudget) return cudaErrorNotSupported;
     }
-    merge_kernel<<<mgrid, kMergeWarps * 32, 0, stream>>>(p, seq_lens, ws, ws.merged, Lc);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // widest dv slice whose W_UV rows fit the shared-memory budget (dv % 8 == 0)
-    int dsub = p.dv;
-    while ((size_t)Lc * dsub * 2 > kWSmemBudget && dsub % 16 == 0) dsub /= 2;
-    const int groups = kProjThreads / dsub;
-    const size_t smem = (size_t)Lc * dsub * 2 + sizeof(float) * ((size_t)kProjChunk * Lc + (size_t)groups * kProjChunk * dsub);
+    const size_t smem = (w_uv ? (size_t)Lc * dsub * 2 + (size_t)kWarps * kRows * dsub * sizeof(float) : 0) +
+                        (size_t)Bc * Lc * sizeof(float);
     constexpr size_t kMaxDyn = 200 * 1024;
     if (smem > kMaxDyn) return cudaErrorNotSupported;
     static unsigned long long attr_done = 0;
-    e = set_smem_once(project_kernel, kMaxDyn, &attr_done);
+    cudaError_t e = set_smem_once(combine_kernel, kMaxDyn, &attr_done);
     if (e != cudaSuccess) return e;
-    dim3 pgrid(p.H, p.dv / dsub);
-    project_kernel<<<pgrid, kProjThreads, smem, stream>>>(p, dsub, w_uv, ws.merged, out);
+    dim3 grid(p.H, w_uv ? p.dv / dsub : 1, (p.B + Bc - 1) / Bc);
+    const uint64_t wait_cycles = 2ull * 1000 * 1000 * 1000;   // about a second at the SM clock
+    combine_kernel<<<grid, kThreads, smem, stream>>>(p, Bc, dsub, seq_lens, ws, w_uv, out, wait_cycles);
     return cudaGetLastError();
 }
 

@@ -43,7 +43,6 @@ struct Plan {
 struct Workspace {
     float* part_lse;   // [slots][H]
     float* part_o;     // [slots][H][Ls]
-    float* merged;     // [B][H][gc * Ls]: merged shard outputs before the W_UV projection
 };
 
 __host__ __device__ inline int num_slots(const Plan& p) { return p.W + p.B * p.gc; }
