@@ -8,13 +8,18 @@
 //     c_s = y_s / sqrt(mean(y_s^2) + eps)  [* w_s]   for every shard s
 // rounded to bf16 (round to nearest even) and written to
 // ckv[page][s][slot][:], with k_pe copied to kpe[page][slot][:].
-// One CTA per new token; this is latency-bound (one token per sequence).
+// One CTA per (new token, shard): the Hadamard transform is computed whole in
+// every shard's CTA (it mixes all L inputs and costs L log L adds), the dense
+// transform only for the shard's L/g rows, four rows per warp at a time so that
+// many loads of R are in flight.  Each CTA normalises and stores its own
+// slice; the shard-0 CTA also copies k_pe.  Latency-bound: one token per
+// sequence.
 #include "tpla_internal.cuh"
 
 namespace tpla {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kMaxL = 1024;
 
 __global__ void __launch_bounds__(kThreads)
@@ -27,17 +32,21 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
     __shared__ float y[kMaxL];
     __shared__ float part[kMaxL / 32];
     __shared__ float inv_rms[8];
-    const int b = blockIdx.x, tid = threadIdx.x;
+    const int b = blockIdx.x, sh = blockIdx.y, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int Ls = L / g;
 
     const int pos = __ldg(positions + b);
     if (pos < 0 || pos >= max_pages * kPage) {
-        if (tid == 0) atomicOr(status, kStatusIndex);
+        if (tid == 0 && sh == 0) atomicOr(status, kStatusIndex);
         return;
     }
-    const int page = page_lookup(block_table, b, pos / kPage, max_pages, num_pages, status);
-    if (page < 0) return;
+    const int lp = pos / kPage;
+    const int page = block_table ? __ldg(block_table + (size_t)b * max_pages + lp) : b * max_pages + lp;
+    if (page < 0 || page >= num_pages) {   // recorded once, by the shard-0 CTA
+        if (tid == 0 && sh == 0) atomicOr(status, kStatusIndex);
+        return;
+    }
     const int slot = pos % kPage;
 
     for (int i = tid; i < L; i += kThreads) x[i] = __bfloat162float(latent_raw[(size_t)b * L + i]);
@@ -59,42 +68,53 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
         const float sc = 1.0f / sqrtf((float)L);
         for (int i = tid; i < L; i += kThreads) y[i] *= sc;
     } else if (transform == TPLA_TRANSFORM_DENSE) {
-        // y_i = sum_j R[i][j] x_j : one warp per output row, coalesced over j
-        for (int i = warp; i < L; i += kThreads / 32) {
-            const float* row = R_dense + (size_t)i * L;
-            float acc = 0.f;
-            for (int j = lane; j < L; j += 32) acc = fmaf(__ldg(row + j), x[j], acc);
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) y[i] = acc;
+        // y_i = sum_j R[i][j] x_j for the shard's rows: each warp takes four rows at a time,
+        // coalesced over j
+        for (int i0 = sh * Ls + warp * 4; i0 < (sh + 1) * Ls; i0 += (kThreads / 32) * 4) {
+            const int nr = min(4, (sh + 1) * Ls - i0);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 16
+            for (int j = lane; j < L; j += 32) {
+                const float xj = x[j];
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    if (r < nr) acc[r] = fmaf(__ldg(R_dense + (size_t)(i0 + r) * L + j), xj, acc[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                for (int o = 16; o > 0; o >>= 1) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
+                if (lane == 0 && r < nr) y[i0 + r] = acc[r];
+            }
         }
     } else {
         for (int i = tid; i < L; i += kThreads) y[i] = x[i];
     }
     __syncthreads();
 
-    // sum of squares per 32-element chunk, then per shard
-    for (int c = warp; c < L / 32; c += kThreads / 32) {
-        float v = y[c * 32 + lane];
+    // sum of squares of this shard's slice: per 32-element chunk, then over the chunks
+    const int y0 = sh * Ls;
+    for (int c = warp; c < Ls / 32; c += kThreads / 32) {
+        float v = y[y0 + c * 32 + lane];
         float ss = v * v;
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         if (lane == 0) part[c] = ss;
     }
     __syncthreads();
-    if (tid < g) {
+    if (tid == 0) {
         float ss = 0.f;
-        for (int c = tid * (Ls / 32); c < (tid + 1) * (Ls / 32); ++c) ss += part[c];
-        inv_rms[tid] = 1.0f / sqrtf(ss / (float)Ls + eps);
+        for (int c = 0; c < Ls / 32; ++c) ss += part[c];
+        inv_rms[0] = 1.0f / sqrtf(ss / (float)Ls + eps);
     }
     __syncthreads();
 
-    for (int i = tid; i < L; i += kThreads) {
-        int s = i / Ls, j = i % Ls;
-        float v = y[i] * inv_rms[s];
-        if (norm_weight) v *= __ldg(norm_weight + i);
-        ckv[(((size_t)page * g + s) * kPage + slot) * Ls + j] = __float2bfloat16_rn(v);
+    for (int j = tid; j < Ls; j += kThreads) {
+        float v = y[y0 + j] * inv_rms[0];
+        if (norm_weight) v *= __ldg(norm_weight + y0 + j);
+        ckv[(((size_t)page * g + sh) * kPage + slot) * Ls + j] = __float2bfloat16_rn(v);
     }
-    for (int r = tid; r < R; r += kThreads)
-        kpe[((size_t)page * kPage + slot) * R + r] = kpe_new[(size_t)b * R + r];
+    if (sh == 0)
+        for (int r = tid; r < R; r += kThreads)
+            kpe[((size_t)page * kPage + slot) * R + r] = kpe_new[(size_t)b * R + r];
 }
 
 }  // namespace
@@ -106,7 +126,7 @@ cudaError_t launch_append(const tpla_dims_t& d, const __nv_bfloat16* latent_raw,
                           unsigned* status, cudaStream_t stream) {
     if (d.B == 0) return cudaSuccess;
     if (d.L > kMaxL) return cudaErrorNotSupported;
-    append_kernel<<<d.B, kThreads, 0, stream>>>(d.L, d.R, d.g, d.max_pages_per_seq, d.num_pages,
+    append_kernel<<<dim3(d.B, d.g), kThreads, 0, stream>>>(d.L, d.R, d.g, d.max_pages_per_seq, d.num_pages,
                                                 latent_raw, kpe_new, transform, R_dense, norm_weight,
                                                 eps, positions, block_table, ckv, kpe, status);
     return cudaGetLastError();

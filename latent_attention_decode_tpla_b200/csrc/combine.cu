@@ -15,9 +15,10 @@
 //      memory (a single copy when the slice is the whole dv);
 //   2. one warp finds, for each (sequence, shard) pair of the group, the
 //      workers holding its first and last tile (a prefix sum over seq_lens);
-//   3. every thread merges one 4-float piece of one pair's row over that
-//      pair's segments in a single pass (running maximum and rescale), so all
-//      partial and log-sum-exp loads are independent;
+//   3. every thread (or group of up to 8 lanes, when there are few pairs)
+//      merges one 4-float piece of one pair's row over that pair's segments
+//      in a single pass (running maximum and rescale), so all partial and
+//      log-sum-exp loads are independent;
 //   4. the projection keeps kRows rows x 8 columns per lane in registers (one
 //      16-byte W_UV load per row of the reduction for 64 FMAs), sums the lanes'
 //      parts by shuffles and the warps' parts through shared memory.
@@ -34,8 +35,9 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr size_t kWSmemBudget = 64 * 1024;     // bytes of W_UV staged per CTA
 constexpr int kMergeTarget = 2048;             // merged floats per CTA the group size aims at
-constexpr int kRows = 8;                       // merged rows projected together
+constexpr int kMaxRows = 8;                    // merged rows projected together, at most
 constexpr int kMaxPairs = 64;                  // (sequence, shard) pairs per CTA
+constexpr int kBatch = 8;                      // segments whose loads a thread issues together
 
 // The schedule's unit boundaries lo(w) = floor(w U / W) and owners, in 32-bit arithmetic when
 // (W + 1) U fits (64-bit integer division is emulated and slow), else in 64 bits.
@@ -56,6 +58,7 @@ struct PairInfo {
     int first_slot;    // slot of the first segment
 };
 
+template <int kRows>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(Plan p, int Bc, int dsub, const int32_t* __restrict__ seq_lens, Workspace ws,
                const __nv_bfloat16* __restrict__ w_uv, float* __restrict__ out, uint64_t wait_cycles) {
@@ -132,33 +135,69 @@ combine_kernel(Plan p, int Bc, int dsub, const int32_t* __restrict__ seq_lens, W
     }
     __syncthreads();
 
-    // 3. merge: one float4 of one pair's row per thread and iteration
+    // 3. merge: one float4 of one pair's row per group of nsplit adjacent lanes; the lanes of a
+    // group take every nsplit-th segment and combine their partial merges by shuffles (when there
+    // are fewer items than threads, e.g. one long sequence split over many workers)
     const int q4 = p.Ls / 4;
-    for (int i = tid; i < npairs * q4; i += kThreads) {
-        const int pr = i / q4, j = (i % q4) * 4;
-        const int bl = pr / p.gc, s = pr % p.gc;
+    const int items = npairs * q4;
+    int nsplit = 1;
+    while (nsplit < 8 && items * nsplit * 2 <= kThreads) nsplit *= 2;
+    const int t = tid % nsplit;
+    for (int base = 0; base < items; base += kThreads / nsplit) {   // same trip count in every lane
+        const int i = base + tid / nsplit;
+        const bool active = i < items;
+        const int pr = active ? i / q4 : 0, j = active ? (i % q4) * 4 : 0;
         const PairInfo pi = pinfo[pr];
         float M = -INFINITY, den = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         // segments: the first one, then one per later worker up to the last.  A worker with an
         // empty range (possible when there are fewer units than workers) left lse = -inf in its
-        // slot, so its weight is 0 and its partial, never written, is not read into the sum.  No
-        // load depends on another, so they are all in flight together.
-#pragma unroll 8
-        for (int k = pi.wf; k <= pi.wl; ++k) {
-            const size_t slot = (size_t)(k == pi.wf ? pi.first_slot : k);
-            const float lse = __ldg(ws.part_lse + slot * p.H + h);
-            float4 v = __ldg(reinterpret_cast<const float4*>(ws.part_o + (slot * p.H + h) * p.Ls + j));
-            const float Mn = fmaxf(M, lse);
-            const float a = exp2f(M - Mn), wk = exp2f(lse - Mn);   // exp2f(-inf) = 0 on the first segment
-            if (wk == 0.f) v = make_float4(0.f, 0.f, 0.f, 0.f);
-            den = den * a + wk;
-            acc.x = acc.x * a + wk * v.x;
-            acc.y = acc.y * a + wk * v.y;
-            acc.z = acc.z * a + wk * v.z;
-            acc.w = acc.w * a + wk * v.w;
+        // slot, so its weight is 0 and its partial, never written, is not read into the sum.  The
+        // loads of a batch of kBatch segments are issued together, then folded in.
+        const int kbeg = active ? pi.wf + t : 1, kend = active ? pi.wl : 0;
+        for (int kb = kbeg; kb <= kend; kb += kBatch * nsplit) {
+            float lse[kBatch];
+            float4 v[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int k = kb + u * nsplit;
+                lse[u] = -INFINITY;
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (k <= kend) {
+                    const size_t slot = (size_t)(k == pi.wf ? pi.first_slot : k);
+                    lse[u] = __ldg(ws.part_lse + slot * p.H + h);
+                    v[u] = __ldg(reinterpret_cast<const float4*>(ws.part_o + (slot * p.H + h) * p.Ls + j));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                if (lse[u] == -INFINITY) continue;
+                const float Mn = fmaxf(M, lse[u]);
+                const float a = exp2f(M - Mn), wk = exp2f(lse[u] - Mn);   // exp2f(-inf) = 0 on the first one
+                den = den * a + wk;
+                acc.x = acc.x * a + wk * v[u].x;
+                acc.y = acc.y * a + wk * v[u].y;
+                acc.z = acc.z * a + wk * v[u].z;
+                acc.w = acc.w * a + wk * v[u].w;
+                M = Mn;
+            }
+        }
+        for (int off = 1; off < nsplit; off <<= 1) {   // combine the group's partial merges
+            const float Mo = __shfl_xor_sync(0xffffffffu, M, off);
+            const float dno = __shfl_xor_sync(0xffffffffu, den, off);
+            const float4 ao = make_float4(__shfl_xor_sync(0xffffffffu, acc.x, off), __shfl_xor_sync(0xffffffffu, acc.y, off),
+                                          __shfl_xor_sync(0xffffffffu, acc.z, off), __shfl_xor_sync(0xffffffffu, acc.w, off));
+            const float Mn = fmaxf(M, Mo);
+            const float e1 = M == -INFINITY ? 0.f : exp2f(M - Mn), e2 = Mo == -INFINITY ? 0.f : exp2f(Mo - Mn);
+            den = den * e1 + dno * e2;
+            acc.x = acc.x * e1 + ao.x * e2;
+            acc.y = acc.y * e1 + ao.y * e2;
+            acc.z = acc.z * e1 + ao.z * e2;
+            acc.w = acc.w * e1 + ao.w * e2;
             M = Mn;
         }
+        if (!active || t != 0) continue;
+        const int bl = pr / p.gc, s = pr % p.gc;
         const float inv = pi.wl >= pi.wf ? 1.0f / den : 0.f;
         const float4 r = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
         if (project) {
@@ -244,11 +283,17 @@ cudaError_t launch_combine(const Plan& p, const int32_t* seq_lens, const __nv_bf
                            float* out, Workspace ws, cudaStream_t stream) {
     if (p.B == 0) return cudaSuccess;
     const int Lc = p.gc * p.Ls;
-    // sequences per CTA: about kMergeTarget merged floats per CTA, whole row chunks when projecting
+    // sequences per CTA: about kMergeTarget merged floats per CTA; when projecting, a power of two
+    // up to kMaxRows, or whole chunks of kMaxRows rows
     int Bc = kMergeTarget / Lc;
     Bc = Bc < 1 ? 1 : (Bc > p.B ? p.B : Bc);
-    if (w_uv) Bc = (Bc + kRows - 1) / kRows * kRows;
-    while (Bc * p.gc > kMaxPairs) Bc = Bc > kRows ? Bc - kRows : Bc / 2;
+    int rows = kMaxRows;
+    if (w_uv) {
+        rows = 1;
+        while (rows < Bc && rows < kMaxRows) rows *= 2;
+        Bc = (Bc + rows - 1) / rows * rows;
+    }
+    while (Bc * p.gc > kMaxPairs) Bc = Bc > rows ? Bc - rows : Bc / 2;
     if (Bc < 1) return cudaErrorNotSupported;
     // dv slice: the widest 8 * 2^k columns (at most 256) that divide dv and whose W_UV rows fit the
     // shared-memory budget (dv % 8 == 0)
@@ -257,17 +302,25 @@ cudaError_t launch_combine(const Plan& p, const int32_t* seq_lens, const __nv_bf
         while (dsub * 2 <= 256 && p.dv % (dsub * 2) == 0 && (size_t)Lc * dsub * 4 <= kWSmemBudget) dsub *= 2;
         if ((size_t)Lc * dsub * 2 > kWSmemBudget) return cudaErrorNotSupported;
     }
-    const size_t smem = (w_uv ? (size_t)Lc * dsub * 2 + (size_t)kWarps * kRows * dsub * sizeof(float) : 0) +
+    const size_t smem = (w_uv ? (size_t)Lc * dsub * 2 + (size_t)kWarps * rows * dsub * sizeof(float) : 0) +
                         (size_t)Bc * Lc * sizeof(float);
     constexpr size_t kMaxDyn = 200 * 1024;
     if (smem > kMaxDyn) return cudaErrorNotSupported;
-    static unsigned long long attr_done = 0;
-    cudaError_t e = set_smem_once(combine_kernel, kMaxDyn, &attr_done);
-    if (e != cudaSuccess) return e;
     dim3 grid(p.H, w_uv ? p.dv / dsub : 1, (p.B + Bc - 1) / Bc);
     const uint64_t wait_cycles = 2ull * 1000 * 1000 * 1000;   // about a second at the SM clock
-    combine_kernel<<<grid, kThreads, smem, stream>>>(p, Bc, dsub, seq_lens, ws, w_uv, out, wait_cycles);
-    return cudaGetLastError();
+    auto launch = [&](auto kern, unsigned long long* done) -> cudaError_t {
+        cudaError_t e = set_smem_once(kern, kMaxDyn, done);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kThreads, smem, stream>>>(p, Bc, dsub, seq_lens, ws, w_uv, out, wait_cycles);
+        return cudaGetLastError();
+    };
+    static unsigned long long done[4] = {0, 0, 0, 0};
+    switch (rows) {
+        case 1: return launch(combine_kernel<1>, &done[0]);
+        case 2: return launch(combine_kernel<2>, &done[1]);
+        case 4: return launch(combine_kernel<4>, &done[2]);
+        default: return launch(combine_kernel<8>, &done[3]);
+    }
 }
 
 }  // namespace tpla
