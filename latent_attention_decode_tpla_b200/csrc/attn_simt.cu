@@ -97,22 +97,29 @@ attn_simt_kernel(Plan p, const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
             }
         }
         __syncthreads();
-        // scores (log2 domain): s = (scale*log2e) * (q . [c | k_pe])
-        for (int i = tid; i < kHG * kPage; i += kThreads) {
-            int h = i / kPage, t = i % kPage;
-            float s = -INFINITY;
-            if (t < valid) {
-                const __nv_bfloat162* row = reinterpret_cast<const __nv_bfloat162*>(&sm.c[t][0]);
-                float d0 = 0.f, d1 = 0.f;
-#pragma unroll 8
-                for (int k = 0; k < K / 2; ++k) {
-                    float2 cv = __bfloat1622float2(row[k]);
-                    d0 = fmaf(sm.q[h][2 * k], cv.x, d0);
-                    d1 = fmaf(sm.q[h][2 * k + 1], cv.y, d1);
+        // scores (log2 domain): s = (scale*log2e) * (q . [c | k_pe]); each thread takes the
+        // kSc (head, token) pairs tid + kThreads * i with the same token t, interleaved
+        {
+            constexpr int kSc = kHG * kPage / kThreads;       // 4
+            static_assert(kHG * kPage % kThreads == 0 && kThreads % kPage == 0, "score map");
+            const int t = tid % kPage, hb = tid / kPage;      // heads hb + (kThreads / kPage) * i
+            const __nv_bfloat162* row = reinterpret_cast<const __nv_bfloat162*>(&sm.c[t][0]);
+            float d0[kSc], d1[kSc];
+#pragma unroll
+            for (int i = 0; i < kSc; ++i) d0[i] = d1[i] = 0.f;
+#pragma unroll 4
+            for (int k = 0; k < K / 2; ++k) {
+                const float2 cv = __bfloat1622float2(row[k]);
+#pragma unroll
+                for (int i = 0; i < kSc; ++i) {
+                    const int h = hb + (kThreads / kPage) * i;
+                    d0[i] = fmaf(sm.q[h][2 * k], cv.x, d0[i]);
+                    d1[i] = fmaf(sm.q[h][2 * k + 1], cv.y, d1[i]);
                 }
-                s = d0 + d1;
             }
-            sm.p[h][t] = s;
+#pragma unroll
+            for (int i = 0; i < kSc; ++i)
+                sm.p[hb + (kThreads / kPage) * i][t] = t < valid ? d0[i] + d1[i] : -INFINITY;
         }
         __syncthreads();
         // online softmax, one warp per head
@@ -135,15 +142,20 @@ attn_simt_kernel(Plan p, const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
             }
         }
         __syncthreads();
-        // o = alpha * o + P C
+        // o = alpha * o + P C, with the token loop outside so that the NACC accumulators give
+        // independent FMAs (rows past `valid` have p = 0 and zeroed cache rows)
 #pragma unroll
         for (int a = 0; a < NACC; ++a) {
-            int flat = tid + kThreads * a;
-            int h = flat / LS, j = flat % LS;
-            if (h < kHG) {
-                float o = acc[a] * sm.alpha[h];
-                for (int t = 0; t < valid; ++t) o = fmaf(sm.p[h][t], __bfloat162float(sm.c[t][j]), o);
-                acc[a] = o;
+            const int flat = tid + kThreads * a;
+            const int h = flat / LS;
+            if (h < kHG) acc[a] *= sm.alpha[h];
+        }
+        for (int t = 0; t < kPage; ++t) {
+#pragma unroll
+            for (int a = 0; a < NACC; ++a) {
+                const int flat = tid + kThreads * a;
+                const int h = flat / LS, j = flat % LS;
+                if (h < kHG) acc[a] = fmaf(sm.p[h][t], __bfloat162float(sm.c[t][j]), acc[a]);
             }
         }
         if (seg_end) {
