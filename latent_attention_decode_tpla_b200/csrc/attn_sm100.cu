@@ -516,56 +516,19 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 for (int k = 4; k < kCols; ++k) e4[k & 3] = fmaxf(e4[k & 3], s[k]);
                 ext = fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]));
             }
-            bars.xmax_buf[j & 1][wg][row] = ext;
+            // Reference maximum of this tile's exponentials, decided without waiting for the other
+            // warpgroup: the running maximum m, raised to this warpgroup's own maximum when that
+            // exceeds m by more than the threshold (always on a segment's first tile).  The raised
+            // references are exchanged after P is formed; the row's new running maximum is the
+            // largest of m and them, and a warpgroup whose reference is below it scales its P down.
+            const float m_loc = ext * sc;                                   // -inf: no valid column
+            const bool raise = warp_active && m_loc > -INFINITY && (first_tile || m_loc > m + kRescaleThreshold);
+            const float m_ref = raise ? m_loc : (m > -INFINITY ? m : 0.f);  // 0: no valid column yet, P = 0
+            bars.xmax_buf[j & 1][wg][row] = raise ? m_loc : -INFINITY;
             warp_arrive(smem_addr(&bars.xmax));
-            if (!wt.wait(smem_addr(&bars.xmax), (uint32_t)(j & 1))) break;
-            const float other = bars.xmax_buf[j & 1][wg ^ 1][row];
-            const float mt = fmaxf(ext, other) * sc;   // max of scale*s
-
-            bool alive = true;
-            if (warp_active) {
-                if (first_tile) {
-                    m = mt;
-                } else {
-                    const bool need = mt > m + kRescaleThreshold;
-                    if (__any_sync(0xffffffffu, need)) {
-                        const float m_use = need ? mt : m;
-                        const float alpha = ex2_approx(m - m_use);
-                        if (!wait_o(j - 1)) alive = false;
-                        if (alive) {
-#pragma unroll 1
-                            for (int c = 0; c < kOHalf / 32; ++c) {
-                                const uint32_t ta = lane_base + C::kColO + wg * kOHalf + c * 32;
-                                uint32_t r[32];
-                                tmem_ld32(ta, r);
-                                tmem_wait_ld();
-#pragma unroll
-                                for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-                                tmem_st32(ta, r);
-                            }
-                            tmem_wait_st();
-                            l *= alpha;
-                            m = m_use;
-                        }
-                    }
-                }
-            }
-            if (!alive) break;
             uint32_t pk[kCols / 2];
-            if (warp_active) {
-                const float nm = -m;
-                // even columns on the special-function unit, odd columns on the FMA pipe
-#pragma unroll
-                for (int k = 0; k < kCols; ++k)
-                    s[k] = ex2_approx(fmaf(s[k], sc, nm));
-                if (tail) {
-#pragma unroll
-                    for (int k = 0; k < kCols; ++k) s[k] = wg * kCols + k < valid ? s[k] : 0.f;
-                }
-                float l4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int k = 0; k < kCols; ++k) l4[k & 3] += s[k];
-                l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            float lt = 0.f;
+            auto pack = [&]() {
                 if (exact) {
 #pragma unroll
                     for (int k = 0; k < kCols / 2; ++k) pk[k] = pack_f16x2(s[2 * k], s[2 * k + 1]);
@@ -573,6 +536,20 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
 #pragma unroll
                     for (int k = 0; k < kCols / 2; ++k) pk[k] = pack_bf16x2(s[2 * k], s[2 * k + 1]);
                 }
+            };
+            if (warp_active) {
+                const float nm = -m_ref;
+#pragma unroll
+                for (int k = 0; k < kCols; ++k) s[k] = ex2_approx(fmaf(s[k], sc, nm));
+                if (tail) {
+#pragma unroll
+                    for (int k = 0; k < kCols; ++k) s[k] = wg * kCols + k < valid ? s[k] : 0.f;
+                }
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int k = 0; k < kCols; ++k) l4[k & 3] += s[k];
+                lt = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                pack();
             } else {
 #pragma unroll
                 for (int k = 0; k < kCols / 2; ++k) pk[k] = 0u;
@@ -605,6 +582,43 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                     const int c = i / (rows * 8), rr = valid + (i / 8) % rows, seg16 = i % 8;
                     *reinterpret_cast<uint4*>(sb + c * C::kChunk + rr * 128 + seg16 * 16) = make_uint4(0, 0, 0, 0);
                 }
+            }
+            // the other warpgroup's raised reference, the row's new running maximum, and the rescales
+            if (!wt.wait(smem_addr(&bars.xmax), (uint32_t)(j & 1))) break;
+            {
+                const float other = bars.xmax_buf[j & 1][wg ^ 1][row];
+                const float m_new = fmaxf(m, fmaxf(raise ? m_loc : -INFINITY, other));
+                bool alive = true;
+                if (warp_active) {
+                    if (__any_sync(0xffffffffu, m_new > m_ref)) {   // P was formed against a lower reference
+                        const float f = m_new > m_ref ? ex2_approx(m_ref - m_new) : 1.0f;
+#pragma unroll
+                        for (int k = 0; k < kCols; ++k) s[k] *= f;
+                        lt *= f;
+                        pack();
+                    }
+                    if (!first_tile && __any_sync(0xffffffffu, m_new > m)) {   // O and l were against m
+                        const float alpha = m_new > m ? ex2_approx(m - m_new) : 1.0f;
+                        if (!wait_o(j - 1)) alive = false;
+                        if (alive) {
+#pragma unroll 1
+                            for (int c = 0; c < kOHalf / 32; ++c) {
+                                const uint32_t ta = lane_base + C::kColO + wg * kOHalf + c * 32;
+                                uint32_t r[32];
+                                tmem_ld32(ta, r);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+                                tmem_st32(ta, r);
+                            }
+                            tmem_wait_st();
+                            l *= alpha;
+                        }
+                    }
+                    m = m_new;
+                    l += lt;
+                }
+                if (!alive) break;
             }
             // the P buffer is free once PV(j - 1), its last reader, has completed
             if (j >= 1 && !wait_o(j - 1)) break;
