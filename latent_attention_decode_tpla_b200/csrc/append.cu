@@ -35,6 +35,9 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
     const int b = blockIdx.x, sh = blockIdx.y, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int Ls = L / g;
+    // the cache this kernel writes may still be read by the previous kernel (an attention pass)
+    pdl_wait();
+    pdl_trigger();
 
     const int pos = __ldg(positions + b);
     if (pos < 0 || pos >= max_pages * kPage) {
@@ -126,10 +129,9 @@ cudaError_t launch_append(const tpla_dims_t& d, const __nv_bfloat16* latent_raw,
                           unsigned* status, cudaStream_t stream) {
     if (d.B == 0) return cudaSuccess;
     if (d.L > kMaxL) return cudaErrorNotSupported;
-    append_kernel<<<dim3(d.B, d.g), kThreads, 0, stream>>>(d.L, d.R, d.g, d.max_pages_per_seq, d.num_pages,
-                                                latent_raw, kpe_new, transform, R_dense, norm_weight,
-                                                eps, positions, block_table, ckv, kpe, status);
-    return cudaGetLastError();
+    return launch_pdl(append_kernel, dim3(d.B, d.g), dim3(kThreads), 0, stream, d.L, d.R, d.g, d.max_pages_per_seq,
+                      d.num_pages, latent_raw, kpe_new, transform, R_dense, norm_weight, eps, positions,
+                      block_table, ckv, kpe, status);
 }
 
 }  // namespace tpla

@@ -47,6 +47,9 @@ attn_simt_kernel(Plan p, const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     const int warp = tid >> 5, lane = tid & 31;
     const int w = blockIdx.x;
     const int h0 = blockIdx.y * kHG;
+    // the cache may have just been written by an append pass; the next kernel launches when the
+    // CTAs of this one have exited (no early trigger)
+    pdl_wait();
 
     const long long U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
     if (U == 0) return;
@@ -187,8 +190,7 @@ cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16*
     cudaError_t e = set_smem_once(kern, smem, &attr_done);
     if (e != cudaSuccess) return e;
     dim3 grid(p.W, (p.H + kHG - 1) / kHG);
-    kern<<<grid, kThreads, smem, stream>>>(p, q, q_pe, ckv, kpe, bt, seq_lens, ws);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(kThreads), smem, stream, p, q, q_pe, ckv, kpe, bt, seq_lens, ws);
 }
 
 template <int LS>

@@ -203,18 +203,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int w = blockIdx.x;
 
-    // every warp derives the same unit range from seq_lens
-    const long long U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
-    if (U == 0) return;
-    const long long lo = unit_lo(w, U, p.W), hi = unit_lo(w + 1, U, p.W);
-    if (lo >= hi) {
-        // a worker with no units leaves a zero-weight partial in its slot: the merge may count it
-        // as a segment of the pair it falls inside
-        for (int i = threadIdx.x; i < p.H; i += blockDim.x) ws.part_lse[(size_t)w * p.H + i] = -INFINITY;
-        return;
-    }
-    const UnitPos pos0 = warp_locate_unit(seq_lens, p.B, p.max_pages, p.gc, lo);
-
+    // barriers first: this part touches no global memory and may overlap the previous kernel
     if (threadIdx.x == 0) {
         for (int i = 0; i < NST; ++i) {
             mbar_init(smem_addr(&bars.full[i]), 1);
@@ -233,7 +222,24 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         bars.abort = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
+        prefetch_tensor_map(&tm_c);
+        prefetch_tensor_map(&tm_k);
     }
+    // every input may have been written by the previous kernel on the stream: wait for it
+    pdl_wait();
+
+    // every warp derives the same unit range from seq_lens
+    const long long U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
+    if (U == 0) return;
+    const long long lo = unit_lo(w, U, p.W), hi = unit_lo(w + 1, U, p.W);
+    if (lo >= hi) {
+        // a worker with no units leaves a zero-weight partial in its slot: the merge may count it
+        // as a segment of the pair it falls inside
+        for (int i = threadIdx.x; i < p.H; i += blockDim.x) ws.part_lse[(size_t)w * p.H + i] = -INFINITY;
+        return;
+    }
+    const UnitPos pos0 = warp_locate_unit(seq_lens, p.B, p.max_pages, p.gc, lo);
+
     if (warp == 1) {
         tmem_alloc(smem_addr(&bars.tmem_base), C::kTmemCols);
         tmem_relinquish();
@@ -248,27 +254,37 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // page-table entries are loaded kPageAhead units ahead of their TMA issue
+            // Page-table entries are loaded kPageAhead units ahead of their TMA issue, as plain
+            // loads that can all be in flight at once; an entry is checked when it is used.
             UnitPos ahead = pos0;
             long long ua = lo;
+            auto raw_page = [&](const UnitPos& u) -> int {
+                return block_table ? __ldg(block_table + (size_t)u.b * p.max_pages + u.tile)
+                                   : u.b * p.max_pages + u.tile;
+            };
             int pg[kPageAhead];
 #pragma unroll
             for (int k = 0; k < kPageAhead; ++k) {
                 pg[k] = -1;
                 if (ua < hi) {
-                    pg[k] = page_lookup(block_table, ahead.b, ahead.tile, p.max_pages, p.num_pages, p.status);
+                    pg[k] = raw_page(ahead);
                     advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
                     ++ua;
                 }
             }
+            // every popped entry belongs to a unit of the range: an entry outside [0, num_pages)
+            // is a caller error, recorded, and the page reads as zeros
             auto pop_page = [&]() -> int {
-                const int page = pg[0];
+                int page = pg[0];
+                if (page < 0 || page >= p.num_pages) {
+                    atomicOr(p.status, kStatusIndex);
+                    page = -1;
+                }
 #pragma unroll
                 for (int k = 0; k + 1 < kPageAhead; ++k) pg[k] = pg[k + 1];
                 pg[kPageAhead - 1] = -1;
                 if (ua < hi) {
-                    pg[kPageAhead - 1] =
-                        page_lookup(block_table, ahead.b, ahead.tile, p.max_pages, p.num_pages, p.status);
+                    pg[kPageAhead - 1] = raw_page(ahead);
                     advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
                     ++ua;
                 }
@@ -283,6 +299,13 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 const int page1 = t.npages == 2 ? pop_page() : -1;
                 if (use > 0 && !wt.wait(smem_addr(&bars.empty[st]), (use - 1) & 1)) break;
                 const int shard = p.shard0 + t.pos.s;
+                if (t.begin && j > 0) {
+                    // the softmax warps load this segment's query when the previous segment's last
+                    // tile is done, a few tiles from now: have it in L2 by then
+                    const __nv_bfloat16* qrow = q + (size_t)t.pos.b * p.H * p.L + (size_t)shard * LS;
+                    for (int h = 0; h < p.H; ++h) prefetch_l2(qrow + (size_t)h * p.L, LS * 2);
+                    prefetch_l2(q_pe + (size_t)t.pos.b * p.H * RD, (uint32_t)(p.H * RD * 2));
+                }
                 const uint32_t full = smem_addr(&bars.full[st]);
                 const uint32_t dst = stage0 + st * C::kStageBytes;
                 mbar_arrive_expect_tx(full, C::kStageBytes);
@@ -299,6 +322,10 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 }
                 t = next_tile(t, seq_lens, p, lo, hi);
             }
+            // All loads are issued: the next kernel (the combine) may launch once every CTA is
+            // here.  Triggering at the start instead lets its CTAs pile onto the SMs whose workers
+            // finish first, which unbalances the combine.
+            pdl_trigger();
             // drain: the last use of every stage must have landed before the CTA exits
             for (long long x = j - NST < 0 ? 0 : j - NST; x < j; ++x) {
                 const int st = (int)(x % NST);
@@ -434,44 +461,65 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             tc_fence_after();
             return true;
         };
-        Tile t = make_tile(pos0, lo, lo, hi);
-        long long j = 0;
-        for (; t.u < hi; ++j) {
-            const UnitPos pos = t.pos;
-            const int shard = p.shard0 + pos.s;
-            if (t.begin) {
-                ++seg;
-                // query of this (b, shard): the latent part into tensor memory as bf16 pairs
-                // (warpgroups take alternate 64-element chunks), the RoPE part into shared memory
-                if (warp_active) {
-                    const uint4* qs = reinterpret_cast<const uint4*>(q + ((size_t)pos.b * p.H + row) * p.L +
-                                                                     (size_t)shard * LS);
+        // Query of one (b, shard) segment: the latent part into tensor memory as bf16 pairs (the
+        // warpgroups take alternate 64-element chunks), the RoPE part into shared memory.  All
+        // global loads are issued before the first store.  Called for the worker's first segment
+        // here, and for each later one as soon as the previous segment's last S has been read
+        // (its last QK^T, the final reader of both, has completed), ahead of that segment's
+        // epilogue, so that the next QK^T overlaps it.
+        auto load_q = [&](const UnitPos& qp) {
+            constexpr int kQc = (C::kChunksC + 1) / 2;    // latent chunks per warpgroup
+            const int shard = p.shard0 + qp.s;
+            if (warp_active) {
+                const uint4* qs = reinterpret_cast<const uint4*>(q + ((size_t)qp.b * p.H + row) * p.L +
+                                                                 (size_t)shard * LS);
+                const uint4* qpp = reinterpret_cast<const uint4*>(q_pe + ((size_t)qp.b * p.H + row) * RD);
+                uint4 x[kQc][8], xp[4];
 #pragma unroll
-                    for (int c = wg; c < C::kChunksC; c += 2) {
+                for (int i = 0; i < kQc; ++i) {
+                    const int c = wg + 2 * i;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        x[i][v] = (row_active && c < C::kChunksC) ? __ldg(qs + c * 8 + v) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) xp[k] = row_active ? __ldg(qpp + wg * 4 + k) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int i = 0; i < kQc; ++i) {
+                    const int c = wg + 2 * i;
+                    if (c < C::kChunksC) {
                         uint32_t r[32];
 #pragma unroll
                         for (int v = 0; v < 8; ++v) {
-                            uint4 x = make_uint4(0, 0, 0, 0);
-                            if (row_active) x = __ldg(qs + c * 8 + v);
-                            r[4 * v + 0] = x.x ^ qflip; r[4 * v + 1] = x.y ^ qflip; r[4 * v + 2] = x.z ^ qflip; r[4 * v + 3] = x.w ^ qflip;
+                            r[4 * v + 0] = x[i][v].x ^ qflip; r[4 * v + 1] = x[i][v].y ^ qflip;
+                            r[4 * v + 2] = x[i][v].z ^ qflip; r[4 * v + 3] = x[i][v].w ^ qflip;
                         }
                         tmem_st32(lane_base + C::kColQ + c * 32, r);
                     }
-                    tmem_wait_st();
                 }
-                {
-                    const uint4* qp = reinterpret_cast<const uint4*>(q_pe + ((size_t)pos.b * p.H + row) * RD);
+                tmem_wait_st();
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int c = wg * 4 + k;
-                        const uint4 x = row_active ? __ldg(qp + c) : make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4*>(qpe_smem + sw128_offset(row, c)) = make_uint4(x.x ^ qflip, x.y ^ qflip, x.z ^ qflip, x.w ^ qflip);
-                    }
-                    fence_proxy_async_smem();
-                }
+                for (int k = 0; k < 4; ++k)
+                    *reinterpret_cast<uint4*>(qpe_smem + sw128_offset(row, wg * 4 + k)) =
+                        make_uint4(xp[k].x ^ qflip, xp[k].y ^ qflip, xp[k].z ^ qflip, xp[k].w ^ qflip);
+            } else {
+                // rows past H: zero RoPE query (the latent columns of these lanes are never read)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    *reinterpret_cast<uint4*>(qpe_smem + sw128_offset(row, wg * 4 + k)) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            warp_arrive(smem_addr(&bars.q_full));
+        };
+        Tile t = make_tile(pos0, lo, lo, hi);
+        load_q(pos0);
+        long long j = 0;
+        for (; t.u < hi; ++j) {
+            const UnitPos pos = t.pos;
+            if (t.begin) {
+                ++seg;
                 if (wg == 0 && lane == 0) (void)effective_len(seq_lens, pos.b, p.max_pages, p.status);
-                tc_fence_before();
-                warp_arrive(smem_addr(&bars.q_full));
                 m = -INFINITY;
                 l = 0.f;
                 first_tile = true;
@@ -633,7 +681,9 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             warp_arrive(smem_addr(&bars.p_full));
             first_tile = false;
 
+            const Tile tn = next_tile(t, seq_lens, p, lo, hi);
             if (t.end) {
+                if (tn.u < hi) load_q(tn.pos);
                 if (!wait_o(j)) break;
                 // the two warpgroups' halves of the softmax sum
                 bars.xsum_buf[seg & 1][wg][row] = l;
@@ -665,7 +715,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 tc_fence_before();
                 warp_arrive(smem_addr(&bars.o_free));
             }
-            t = next_tile(t, seq_lens, p, lo, hi);
+            t = tn;
         }
     }
 
@@ -724,8 +774,8 @@ cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16*
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_once(kern, smem, &attr_done);
     if (e != cudaSuccess) return e;
-    kern<<<p.W, kThreads, smem, stream>>>(tc, tk, p, q, q_pe, bt, seq_lens, ws, wait_ns, debug_stall);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(p.W), dim3(kThreads), smem, stream, tc, tk, p, q, q_pe, bt, seq_lens, ws, wait_ns,
+                      debug_stall);
 }
 
 }  // namespace

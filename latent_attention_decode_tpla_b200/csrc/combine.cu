@@ -134,6 +134,10 @@ combine_kernel(Plan p, int Bc, int dsub, const int32_t* __restrict__ seq_lens, W
         }
     }
     __syncthreads();
+    // the partials come from the previous grid (the attention pass of this call): wait for it, then
+    // let the next kernel launch
+    pdl_wait();
+    pdl_trigger();
 
     // 3. merge: one float4 of one pair's row per group of nsplit adjacent lanes; the lanes of a
     // group take every nsplit-th segment and combine their partial merges by shuffles (when there
@@ -311,8 +315,7 @@ cudaError_t launch_combine(const Plan& p, const int32_t* seq_lens, const __nv_bf
     auto launch = [&](auto kern, unsigned long long* done) -> cudaError_t {
         cudaError_t e = set_smem_once(kern, kMaxDyn, done);
         if (e != cudaSuccess) return e;
-        kern<<<grid, kThreads, smem, stream>>>(p, Bc, dsub, seq_lens, ws, w_uv, out, wait_cycles);
-        return cudaGetLastError();
+        return launch_pdl(kern, grid, dim3(kThreads), smem, stream, p, Bc, dsub, seq_lens, ws, w_uv, out, wait_cycles);
     };
     static unsigned long long done[4] = {0, 0, 0, 0};
     switch (rows) {

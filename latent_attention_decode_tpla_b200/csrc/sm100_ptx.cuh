@@ -74,6 +74,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint
         : "memory");
 }
 
+// Pull a tensor map (a __grid_constant__ kernel parameter) into the descriptor cache ahead of its
+// first use.
+__device__ __forceinline__ void prefetch_tensor_map(const void* tm) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
+}
+
+// Hint: bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // contiguous global -> shared copy of `bytes` (a multiple of 16, both addresses 16-byte aligned),
 // completing on the mbarrier's transaction count
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

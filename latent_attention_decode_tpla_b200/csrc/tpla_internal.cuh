@@ -172,6 +172,38 @@ inline cudaError_t set_smem_once(Kern kern, size_t bytes, unsigned long long* do
     return e;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+//
+// The kernels of a decode step are launched so that each may start while the previous kernel on the
+// stream finishes (its prologue overlaps that kernel's tail).  pdl_wait() returns once the previous
+// grid on the stream has completed and its writes are visible (at once when it was launched normally
+// and has finished); pdl_trigger() lets the next grid launch.  Rules that keep this safe whatever
+// the caller launches around the library:
+//   * every CTA triggers only after its own wait has returned, so when a kernel starts, the kernel
+//     two launches back has completed and everything it or earlier work wrote is visible;
+//   * before its wait a kernel reads only data the immediately preceding kernel cannot write (the
+//     combine, always preceded by the attention pass of the same call, stages W_UV and seq_lens),
+//     and writes nothing to global memory.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch `kern` on `stream` with programmatic stream serialisation allowed.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- launchers (one per .cu file)
 
 cudaError_t launch_attention_simt(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16* q_pe,
