@@ -22,6 +22,10 @@ int g_opt_debug_stall = 0;   // TPLA_OPT_DEBUG_STALL
 int g_last_kernel = 0;       // TPLA_OPT_LAST_ATTENTION_KERNEL
 
 constexpr int kMinUnitsPerWorker = 6;   // keeps partial traffic small at batch 1
+// A worker whose range ends one (sequence, shard) and starts the next stops its stream for the
+// first one's epilogue and the second one's query load: measured on B200 at about as long as
+// this many units of streaming.
+constexpr long long kSwitchUnits = 8;
 
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mutex;
@@ -120,7 +124,16 @@ int make_plan(const tpla_dims_t* d, int shard, Plan* p) {
     if (g_opt_max_workers > 0 && g_opt_max_workers < cap) cap = g_opt_max_workers;
     const long long umax = (long long)p->gc * d->B * d->max_pages_per_seq;
     long long w = (umax + kMinUnitsPerWorker - 1) / kMinUnitsPerWorker;
-    p->W = (int)(w < 1 ? 1 : (w > cap ? cap : w));
+    w = w < 1 ? 1 : (w > cap ? cap : w);
+    // With a multiple of the (sequence, shard) pair count as the worker count, equal-length pairs
+    // split at worker boundaries and no worker switches pairs.  Take it when, for pairs of the
+    // longest length, the longer ranges cost less than one switch.
+    const long long pairs = (long long)p->gc * d->B, n = d->max_pages_per_seq;
+    if (pairs > 1 && pairs <= w) {
+        const long long wa = (w / pairs) * pairs;
+        if (pairs * n * w <= (pairs * n + kSwitchUnits * w) * wa) w = wa;
+    }
+    p->W = (int)w;
     return TPLA_OK;
 }
 

@@ -184,7 +184,8 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
 
 template <int LS, int RD, int NST>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_k, Plan p,
+attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_o, Plan p,
                   const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ q_pe,
                   const int32_t* __restrict__ block_table, const int32_t* __restrict__ seq_lens, Workspace ws,
                   uint64_t wait_ns, int debug_stall) {
@@ -256,6 +257,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         if (lane == 0) {
             // Page-table entries are loaded kPageAhead units ahead of their TMA issue, as plain
             // loads that can all be in flight at once; an entry is checked when it is used.
+            // (Prefetching the units a stage ring ahead into L2 measured slower on B200.)
             UnitPos ahead = pos0;
             long long ua = lo;
             auto raw_page = [&](const UnitPos& u) -> int {
@@ -345,9 +347,12 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         if (lane == 0) {
             bool ok = true;
             if (debug_stall) ok = wt.wait(smem_addr(&bars.never), 0);   // nothing arrives: exercises the time-out
-            // Issue whichever MMA is ready, polling without blocking: QK^T of the next tile as
-            // soon as its stage has landed and S has been read, PV of the oldest tile as soon as
-            // its P is in shared memory.  Each stream has its own tile cursor.
+            // Issue whichever MMA is ready, polling without blocking: PV of the oldest tile as soon
+            // as its P is in shared memory, QK^T of the next tile as soon as its stage has landed
+            // and S has been read.  PV goes first when both are ready, since it releases a stage
+            // for the next load.  (Issuing QK^T in several groups, to let a PV that becomes ready
+            // meanwhile in sooner, measured much slower on B200: the issue of a group costs far
+            // more than its MMAs.)  Each stream has its own tile cursor.
             Tile tq = make_tile(pos0, lo, lo, hi), tv = tq;
             long long jq = 0, jv = 0;
             int qseg = -1, vseg = -1;
@@ -355,32 +360,6 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             long long idle_since = clock64();
             while (ok && tv.u < hi) {
                 bool did = false;
-                if (tq.u < hi) {
-                    const int st = (int)(jq % NST);
-                    if ((!tq.begin || mbar_test_wait(smem_addr(&bars.q_full), (uint32_t)((qseg + 1) & 1))) &&
-                        mbar_test_wait(smem_addr(&bars.full[st]), (uint32_t)((jq / NST) & 1)) &&
-                        (jq == 0 || mbar_test_wait(smem_addr(&bars.s_free), (uint32_t)((jq - 1) & 1)))) {
-                        if (tq.begin) ++qseg;
-                        tc_fence_after();
-                        const uint32_t sb = stage0 + st * C::kStageBytes;
-                        const uint32_t d = tmem + C::kColS;
-#pragma unroll
-                        for (int kk = 0; kk < C::kStepsC; ++kk) {
-                            const uint64_t bd = smem_desc_sw128(sb + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024);
-                            mma_ts(d, tmem + C::kColQ + kk * 8, bd, C::kIdescQK, kk > 0 ? 1u : 0u);
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < C::kStepsR; ++kk) {
-                            const uint64_t ad = smem_desc_sw128(qpe_addr + kk * 32, 16, 1024);
-                            const uint64_t bd = smem_desc_sw128(sb + C::kChunksC * C::kChunk + kk * 32, 16, 1024);
-                            mma_ss(d, ad, bd, C::kIdescQK, 1u);
-                        }
-                        mma_commit(smem_addr(&bars.s_full));
-                        tq = next_tile(tq, seq_lens, p, lo, hi);
-                        ++jq;
-                        did = true;
-                    }
-                }
                 if (jv < jq) {
                     if (tv.begin && !vbegun) {
                         ++vseg;
@@ -406,6 +385,32 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                         tv = next_tile(tv, seq_lens, p, lo, hi);
                         ++jv;
                         vbegun = false;
+                        did = true;
+                    }
+                }
+                if (tq.u < hi) {
+                    const int st = (int)(jq % NST);
+                    if ((!tq.begin || mbar_test_wait(smem_addr(&bars.q_full), (uint32_t)((qseg + 1) & 1))) &&
+                        mbar_test_wait(smem_addr(&bars.full[st]), (uint32_t)((jq / NST) & 1)) &&
+                        (jq == 0 || mbar_test_wait(smem_addr(&bars.s_free), (uint32_t)((jq - 1) & 1)))) {
+                        if (tq.begin) ++qseg;
+                        tc_fence_after();
+                        const uint32_t sb = stage0 + st * C::kStageBytes;
+                        const uint32_t d = tmem + C::kColS;
+#pragma unroll
+                        for (int kk = 0; kk < C::kStepsC; ++kk) {
+                            const uint64_t bd = smem_desc_sw128(sb + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024);
+                            mma_ts(d, tmem + C::kColQ + kk * 8, bd, C::kIdescQK, kk > 0 ? 1u : 0u);
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < C::kStepsR; ++kk) {
+                            const uint64_t ad = smem_desc_sw128(qpe_addr + kk * 32, 16, 1024);
+                            const uint64_t bd = smem_desc_sw128(sb + C::kChunksC * C::kChunk + kk * 32, 16, 1024);
+                            mma_ss(d, ad, bd, C::kIdescQK, 1u);
+                        }
+                        mma_commit(smem_addr(&bars.s_full));
+                        tq = next_tile(tq, seq_lens, p, lo, hi);
+                        ++jq;
                         did = true;
                     }
                 }
@@ -694,22 +699,36 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 const long long seg_first = u_first < lo ? lo : u_first;
                 const int slot = seg_first == lo ? w : p.W + pos.b * p.gc + pos.s;
                 if (warp_active) {
+                    // The normalised rows go out 32 columns at a time: staged in this warp's own
+                    // rows of the P buffer (free: the segment's last PV has completed), 128B-swizzled,
+                    // and written by a TMA store of a 32 x 32 box.  Rows past H lie outside the
+                    // tensor map and are not written.  Each box waits until the previous store has
+                    // read the buffer; the last wait comes before P is written again.
                     const float inv_l = 1.0f / lt;
-                    float4* dst = reinterpret_cast<float4*>(ws.part_o + ((size_t)slot * p.H + row) * LS + wg * kOHalf);
+                    uint8_t* stile = p_smem + wg * C::kPChunk + quad * 4096;
 #pragma unroll 1
                     for (int c = 0; c < kOHalf / 32; ++c) {
                         uint32_t r[32];
                         tmem_ld32(lane_base + C::kColO + wg * kOHalf + c * 32, r);
                         tmem_wait_ld();
-                        if (row_active) {
+                        if (c > 0) {
+                            if (lane == 0) bulk_wait_read_all();
+                            __syncwarp();
+                        }
 #pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                dst[c * 8 + v] = make_float4(__uint_as_float(r[4 * v]) * inv_l,
-                                                             __uint_as_float(r[4 * v + 1]) * inv_l,
-                                                             __uint_as_float(r[4 * v + 2]) * inv_l,
-                                                             __uint_as_float(r[4 * v + 3]) * inv_l);
+                        for (int v = 0; v < 8; ++v)
+                            *reinterpret_cast<float4*>(stile + sw128_offset(lane, v)) =
+                                make_float4(__uint_as_float(r[4 * v]) * inv_l, __uint_as_float(r[4 * v + 1]) * inv_l,
+                                            __uint_as_float(r[4 * v + 2]) * inv_l, __uint_as_float(r[4 * v + 3]) * inv_l);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&tm_o, smem_addr(stile), wg * kOHalf + c * 32, quad * 32, slot);
+                            bulk_commit();
                         }
                     }
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
                     if (row_active && wg == 0) ws.part_lse[(size_t)slot * p.H + row] = m + log2f(lt);
                 }
                 tc_fence_before();
@@ -719,6 +738,8 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         }
     }
 
+    // the partial outputs' TMA stores have completed when the CTA exits
+    if (warp >= kSoftmaxWarp0 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -746,6 +767,20 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// 3-D fp32 tensor map over the partial outputs [slots][H][Ls] with a 32 x 32 x 1 box (32 columns of
+// 32 rows of one slot) and 128-byte swizzle, for the TMA stores of the epilogue
+bool make_map_o(CUtensorMap* m, void* base, uint64_t ls, uint64_t h, uint64_t slots) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {ls, h, slots};
+    cuuint64_t strides[2] = {ls * 4, h * ls * 4};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 tensor map over [rows][cols] with a 64 x 64 box and 128-byte swizzle
 bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
     EncodeTiledFn fn = encode_fn();
@@ -767,6 +802,8 @@ cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16*
     CUtensorMap tc, tk;
     if (!make_map(&tc, ckv, LS, (uint64_t)p.num_pages * p.g * kPage)) return cudaErrorInvalidValue;
     if (!make_map(&tk, kpe, RD, (uint64_t)p.num_pages * kPage)) return cudaErrorInvalidValue;
+    CUtensorMap to;
+    if (!make_map_o(&to, ws.part_o, LS, p.H, (uint64_t)num_slots(p))) return cudaErrorInvalidValue;
     const size_t smem = C::kSmem + sizeof(Bars<NST>);
     static_assert(C::kTmemCols < 512 || C::kSmem > 116 * 1024, "a 512-column TMEM allocation needs one CTA per SM");
     static_assert(C::kSmem + sizeof(Bars<NST>) <= 227 * 1024, "shared memory");
@@ -774,8 +811,8 @@ cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16*
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_once(kern, smem, &attr_done);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(p.W), dim3(kThreads), smem, stream, tc, tk, p, q, q_pe, bt, seq_lens, ws, wait_ns,
-                      debug_stall);
+    return launch_pdl(kern, dim3(p.W), dim3(kThreads), smem, stream, tc, tk, to, p, q, q_pe, bt, seq_lens, ws,
+                      wait_ns, debug_stall);
 }
 
 }  // namespace
