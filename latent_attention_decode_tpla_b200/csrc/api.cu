@@ -21,7 +21,9 @@ int g_opt_wait_limit = 0;    // TPLA_OPT_WAIT_LIMIT
 int g_opt_debug_stall = 0;   // TPLA_OPT_DEBUG_STALL
 int g_last_kernel = 0;       // TPLA_OPT_LAST_ATTENTION_KERNEL
 
-constexpr int kMinUnitsPerWorker = 6;   // keeps partial traffic small at batch 1
+// Fewest units a tcgen05 worker gets: keeps the partial traffic small at batch 1.  The CUDA-core
+// kernel is bound by arithmetic, not by that traffic, and spreads the units as widely as it can.
+constexpr int kMinUnitsPerWorker = 6;
 // A worker whose range ends one (sequence, shard) and starts the next stops its stream for the
 // first one's epilogue and the second one's query load: measured on B200 at about as long as
 // this many units of streaming.
@@ -123,7 +125,8 @@ int make_plan(const tpla_dims_t* d, int shard, Plan* p) {
     int cap = sms < kMaxWorkers ? sms : kMaxWorkers;
     if (g_opt_max_workers > 0 && g_opt_max_workers < cap) cap = g_opt_max_workers;
     const long long umax = (long long)p->gc * d->B * d->max_pages_per_seq;
-    long long w = (umax + kMinUnitsPerWorker - 1) / kMinUnitsPerWorker;
+    const int min_units = sm100_supports(*p) ? kMinUnitsPerWorker : 1;
+    long long w = (umax + min_units - 1) / min_units;
     w = w < 1 ? 1 : (w > cap ? cap : w);
     // With a multiple of the (sequence, shard) pair count as the worker count, equal-length pairs
     // split at worker boundaries and no worker switches pairs.  Take it when, for pairs of the
