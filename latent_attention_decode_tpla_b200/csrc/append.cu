@@ -52,10 +52,41 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
     }
     const int slot = pos % kPage;
 
-    for (int i = tid; i < L; i += kThreads) x[i] = __bfloat162float(latent_raw[(size_t)b * L + i]);
+    float xv = 0.f;                                   // x[tid] when L <= kThreads
+    if (L <= kThreads) {
+        if (tid < L) xv = __bfloat162float(latent_raw[(size_t)b * L + tid]);
+        if (transform != TPLA_TRANSFORM_HADAMARD && tid < L) x[tid] = xv;
+    } else {
+        for (int i = tid; i < L; i += kThreads) x[i] = __bfloat162float(latent_raw[(size_t)b * L + i]);
+    }
     __syncthreads();
 
-    if (transform == TPLA_TRANSFORM_HADAMARD) {
+    if (transform == TPLA_TRANSFORM_HADAMARD && L <= kThreads) {
+        // Radix-2 butterflies over L = 2^k points (Sylvester order), one point per thread: the
+        // pair (i, i + h) of stage h becomes (a + c, a - c).  Strides below 32 pair lanes of one
+        // warp (shuffles); wider strides go through shared memory, alternating two buffers so
+        // that one barrier per stage suffices.  Whole warps are idle when tid >= L (L >= 64).
+        float v = xv;
+        if (tid < L) {
+            for (int h = 1; h < 32 && h < L; h <<= 1) {
+                const float o = __shfl_xor_sync(0xffffffffu, v, h);
+                v = (tid & h) ? o - v : v + o;
+            }
+        }
+        int buf = 0;
+        for (int h = 32; h < L; h <<= 1) {
+            float* yb = buf ? y : x;
+            if (tid < L) yb[tid] = v;
+            __syncthreads();
+            if (tid < L) {
+                const float o = yb[tid ^ h];
+                v = (tid & h) ? o - v : v + o;
+            }
+            buf ^= 1;
+        }
+        __syncthreads();   // every read of the last stage's buffer is done before y is written
+        if (tid < L) y[tid] = v * (1.0f / sqrtf((float)L));
+    } else if (transform == TPLA_TRANSFORM_HADAMARD) {
         // in-place radix-2 butterflies over L = 2^k points (Sylvester order), then 1/sqrt(L)
         for (int i = tid; i < L; i += kThreads) y[i] = x[i];
         __syncthreads();
@@ -72,16 +103,27 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
         for (int i = tid; i < L; i += kThreads) y[i] *= sc;
     } else if (transform == TPLA_TRANSFORM_DENSE) {
         // y_i = sum_j R[i][j] x_j for the shard's rows: each warp takes four rows at a time,
-        // coalesced over j
+        // coalesced over j, with the loads of kDenseBatch columns per row issued together
+        constexpr int kDenseBatch = 16;
         for (int i0 = sh * Ls + warp * 4; i0 < (sh + 1) * Ls; i0 += (kThreads / 32) * 4) {
             const int nr = min(4, (sh + 1) * Ls - i0);
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 16
-            for (int j = lane; j < L; j += 32) {
-                const float xj = x[j];
+            for (int j0 = 0; j0 < L; j0 += 32 * kDenseBatch) {
+                float rv[4][kDenseBatch];
 #pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    if (r < nr) acc[r] = fmaf(__ldg(R_dense + (size_t)(i0 + r) * L + j), xj, acc[r]);
+                for (int u = 0; u < kDenseBatch; ++u) {
+                    const int j = j0 + u * 32 + lane;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        rv[r][u] = (r < nr && j < L) ? __ldg(R_dense + (size_t)(i0 + r) * L + j) : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < kDenseBatch; ++u) {
+                    const int j = j0 + u * 32 + lane;
+                    const float xj = j < L ? x[j] : 0.f;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) acc[r] = fmaf(rv[r][u], xj, acc[r]);
+                }
             }
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
