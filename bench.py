@@ -57,10 +57,19 @@ def algorithmic_bytes(spec, seq_lens_sum, mode):
     return cache, cache + queries
 
 
-def source_digest():
+# sources that decide what one launch of a kernel does (its code, the shared schedule, the host-side plan)
+KERNEL_SOURCES = {
+    "attn_sm100": ["attn_sm100.cu", "sm100_ptx.cuh", "tpla_internal.cuh", "api.cu"],
+}
+
+
+def source_digest(kernel=None):
+    """Digest of the kernel's sources (all of csrc/ when the kernel is not listed)."""
+    csrc = os.path.join(ROOT, "latent_attention_decode_tpla_b200", "csrc")
+    names = KERNEL_SOURCES.get(kernel) or sorted(os.path.basename(f) for f in glob.glob(os.path.join(csrc, "*")))
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "latent_attention_decode_tpla_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for name in names:
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -74,7 +83,7 @@ def profiled_traffic(kernel, workload):
         if ":" in ln:
             k, v = ln.split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("source_digest") != source_digest():
+    if vals.get("source_digest") != source_digest(kernel):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
