@@ -182,7 +182,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
     return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
-template <int LS, int RD, int NST>
+template <int LS, int RD, int NST, bool HALF>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_o, Plan p,
@@ -441,20 +441,28 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         const int sw = warp - kSoftmaxWarp0;              // 0..7
         const int wg = sw >> 2;                           // which half of the tile columns and of O
         const int quad = warp & 3;
-        const int row = quad * 32 + lane;                 // head row == TMEM lane
+        const int row = quad * 32 + lane;                 // TMEM lane (row of S, P, O and the query)
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-        const bool warp_active = quad * 32 < p.H;
-        const bool row_active = row < p.H;
+        // With at most 64 heads (HALF), lanes 64-127 carry the query of lanes 0-63, so their S rows
+        // repeat rows 0-63 at no extra MMA cost, and all eight warps share the softmax: a head's
+        // 128 score columns are split four ways (warpgroup x lower/upper lane half) instead of
+        // two.  P rows 64-127 stay zero, so O rows 64-127 stay zero; only the lower half keeps O.
+        const int hrow = HALF ? (row & 63) : row;         // head of this lane
+        const bool upper = HALF && quad >= 2;
+        const bool warp_active = (HALF ? (quad & 1) * 32 : quad * 32) < p.H;
+        const bool row_active = hrow < p.H;
+        const bool o_warp = warp_active && !upper;        // keeps, rescales and writes O rows
         const int tid_sm = threadIdx.x - kSoftmaxWarp0 * 32;   // 0..255
         // A negative scale is folded into the query: its bf16 sign bits are flipped on load (exact),
         // so the scores this kernel sees are multiplied by |scale| and the row maximum is the max.
         const float sc = fabsf(p.scale_log2);
         const uint32_t qflip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
         constexpr int kOHalf = LS / 2;                    // O columns per warpgroup
-        constexpr int kCols = kTileTok / 2;               // score columns per warpgroup
+        constexpr int kCols = HALF ? kTileTok / 4 : kTileTok / 2;   // score columns per thread
+        const int cbase = wg * (kTileTok / 2) + (upper ? kCols : 0);  // the first of them
         long long last_o = -1;                            // highest PV index whose completion was observed
         int seg = -1;
-        float m = -INFINITY, l = 0.f;                     // l: this warpgroup's half of the row sum
+        float m = -INFINITY, l = 0.f;                     // l: this thread's part of the row sum
         bool first_tile = true;
         bool exact = false;                               // fp16 PV for this segment
         // PV(t) is the t-th completion of o_done; completions are in order, so observing PV(t)
@@ -476,9 +484,9 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             constexpr int kQc = (C::kChunksC + 1) / 2;    // latent chunks per warpgroup
             const int shard = p.shard0 + qp.s;
             if (warp_active) {
-                const uint4* qs = reinterpret_cast<const uint4*>(q + ((size_t)qp.b * p.H + row) * p.L +
+                const uint4* qs = reinterpret_cast<const uint4*>(q + ((size_t)qp.b * p.H + hrow) * p.L +
                                                                  (size_t)shard * LS);
-                const uint4* qpp = reinterpret_cast<const uint4*>(q_pe + ((size_t)qp.b * p.H + row) * RD);
+                const uint4* qpp = reinterpret_cast<const uint4*>(q_pe + ((size_t)qp.b * p.H + hrow) * RD);
                 uint4 x[kQc][8], xp[4];
 #pragma unroll
                 for (int i = 0; i < kQc; ++i) {
@@ -517,6 +525,12 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             tc_fence_before();
             warp_arrive(smem_addr(&bars.q_full));
         };
+        if (HALF && upper) {
+            // P rows 64-127 (this warp's lanes, in its warpgroup's K chunk) stay zero
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<uint4*>(p_smem + wg * C::kPChunk + sw128_offset(row, k)) = make_uint4(0, 0, 0, 0);
+        }
         Tile t = make_tile(pos0, lo, lo, hi);
         load_q(pos0);
         long long j = 0;
@@ -538,14 +552,13 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             tc_fence_after();
             float s[kCols];
             if (warp_active) {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(lane_base + C::kColS + wg * kCols, r0);
-                tmem_ld32(lane_base + C::kColS + wg * kCols + 32, r1);
-                tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    s[k] = __uint_as_float(r0[k]);
-                    s[k + 32] = __uint_as_float(r1[k]);
+                for (int h = 0; h < kCols / 32; ++h) {
+                    uint32_t r[32];
+                    tmem_ld32(lane_base + C::kColS + cbase + 32 * h, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) s[32 * h + k] = __uint_as_float(r[k]);
                 }
             } else {
 #pragma unroll
@@ -560,7 +573,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             if (warp_active) {
                 if (tail) {
 #pragma unroll
-                    for (int k = 0; k < kCols; ++k) s[k] = wg * kCols + k < valid ? s[k] : -INFINITY;
+                    for (int k = 0; k < kCols; ++k) s[k] = cbase + k < valid ? s[k] : -INFINITY;
                 }
                 float e4[4];
 #pragma unroll
@@ -596,7 +609,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 for (int k = 0; k < kCols; ++k) s[k] = ex2_approx(fmaf(s[k], sc, nm));
                 if (tail) {
 #pragma unroll
-                    for (int k = 0; k < kCols; ++k) s[k] = wg * kCols + k < valid ? s[k] : 0.f;
+                    for (int k = 0; k < kCols; ++k) s[k] = cbase + k < valid ? s[k] : 0.f;
                 }
                 float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -639,7 +652,9 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             // the other warpgroup's raised reference, the row's new running maximum, and the rescales
             if (!wt.wait(smem_addr(&bars.xmax), (uint32_t)(j & 1))) break;
             {
-                const float other = bars.xmax_buf[j & 1][wg ^ 1][row];
+                float other = bars.xmax_buf[j & 1][wg ^ 1][row];
+                if (HALF)
+                    other = fmaxf(other, fmaxf(bars.xmax_buf[j & 1][wg][row ^ 64], bars.xmax_buf[j & 1][wg ^ 1][row ^ 64]));
                 const float m_new = fmaxf(m, fmaxf(raise ? m_loc : -INFINITY, other));
                 bool alive = true;
                 if (warp_active) {
@@ -651,9 +666,12 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                         pack();
                     }
                     if (!first_tile && __any_sync(0xffffffffu, m_new > m)) {   // O and l were against m
+                        // (an upper-half warp only rescales its part of l)
                         const float alpha = m_new > m ? ex2_approx(m - m_new) : 1.0f;
-                        if (!wait_o(j - 1)) alive = false;
-                        if (alive) {
+                        if (o_warp && !wait_o(j - 1)) alive = false;
+                        if (!o_warp) {
+                            l *= alpha;
+                        } else if (alive) {
 #pragma unroll 1
                             for (int c = 0; c < kOHalf / 32; ++c) {
                                 const uint32_t ta = lane_base + C::kColO + wg * kOHalf + c * 32;
@@ -676,10 +694,13 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             // the P buffer is free once PV(j - 1), its last reader, has completed
             if (j >= 1 && !wait_o(j - 1)) break;
             {
-                uint8_t* pb = p_smem + wg * C::kPChunk;   // this warpgroup's 64 tokens: one K chunk of P
+                // this warpgroup's 64 tokens are one K chunk of P; this thread's columns are the
+                // 16-byte pieces from (cbase mod 64) / 8 on, in its head's row
+                uint8_t* pb = p_smem + wg * C::kPChunk;
+                const int k0 = upper ? kCols / 8 : 0;
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    *reinterpret_cast<uint4*>(pb + sw128_offset(row, k)) =
+                for (int k = 0; k < kCols / 8; ++k)
+                    *reinterpret_cast<uint4*>(pb + sw128_offset(hrow, k0 + k)) =
                         make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
             }
             fence_proxy_async_smem();
@@ -694,11 +715,12 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 bars.xsum_buf[seg & 1][wg][row] = l;
                 warp_arrive(smem_addr(&bars.xsum));
                 if (!wt.wait(smem_addr(&bars.xsum), (uint32_t)(seg & 1))) break;
-                const float lt = l + bars.xsum_buf[seg & 1][wg ^ 1][row];
+                float lt = l + bars.xsum_buf[seg & 1][wg ^ 1][row];
+                if (HALF) lt += bars.xsum_buf[seg & 1][wg][row ^ 64] + bars.xsum_buf[seg & 1][wg ^ 1][row ^ 64];
                 const long long u_first = t.u - pos.tile;       // unit of page 0 of this (b, s)
                 const long long seg_first = u_first < lo ? lo : u_first;
                 const int slot = seg_first == lo ? w : p.W + pos.b * p.gc + pos.s;
-                if (warp_active) {
+                if (o_warp) {
                     // The normalised rows go out 32 columns at a time: staged in this warp's own
                     // rows of the P buffer (free: the segment's last PV has completed), 128B-swizzled,
                     // and written by a TMA store of a 32 x 32 box.  Rows past H lie outside the
@@ -794,7 +816,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int LS, int RD, int NST>
+template <int LS, int RD, int NST, bool HALF>
 cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16* q_pe, const __nv_bfloat16* ckv,
                      const __nv_bfloat16* kpe, const int32_t* bt, const int32_t* seq_lens, Workspace ws,
                      uint64_t wait_ns, int debug_stall, cudaStream_t stream) {
@@ -807,7 +829,7 @@ cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16*
     const size_t smem = C::kSmem + sizeof(Bars<NST>);
     static_assert(C::kTmemCols < 512 || C::kSmem > 116 * 1024, "a 512-column TMEM allocation needs one CTA per SM");
     static_assert(C::kSmem + sizeof(Bars<NST>) <= 227 * 1024, "shared memory");
-    auto kern = attn_sm100_kernel<LS, RD, NST>;
+    auto kern = attn_sm100_kernel<LS, RD, NST, HALF>;
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_once(kern, smem, &attr_done);
     if (e != cudaSuccess) return e;
@@ -826,11 +848,18 @@ cudaError_t launch_attention_sm100(const Plan& p, const __nv_bfloat16* q, const 
                                    const int32_t* block_table, const int32_t* seq_lens, Workspace ws,
                                    int wait_limit_us, int debug_stall, cudaStream_t stream) {
     const uint64_t wait_ns = (wait_limit_us > 0 ? (uint64_t)wait_limit_us : 1000000ull) * 1000ull;
+    const bool half = p.H <= 64;
+#define TPLA_LAUNCH(LS, NST)                                                                                       \
+    return half ? launch_t<LS, 64, NST, true>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, \
+                                              stream)                                                              \
+                : launch_t<LS, 64, NST, false>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, \
+                                               stream)
     switch (p.Ls) {
-        case 256: return launch_t<256, 64, 2>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
-        case 128: return launch_t<128, 64, 3>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
-        case 64: return launch_t<64, 64, 5>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, stream);
+        case 256: TPLA_LAUNCH(256, 2);
+        case 128: TPLA_LAUNCH(128, 3);
+        case 64: TPLA_LAUNCH(64, 5);
     }
+#undef TPLA_LAUNCH
     return cudaErrorNotSupported;
 }
 

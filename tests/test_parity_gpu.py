@@ -69,6 +69,7 @@ RAGGED = [0, 1, 63, 64, 65, 200, 7, 129]
 @pytest.mark.parametrize("H,L,R,dv,g", [
     (8, 64, 16, 32, 2), (128, 512, 64, 128, 1), (128, 512, 64, 128, 2), (64, 512, 64, 128, 4),
     (100, 512, 64, 128, 2), (128, 512, 64, 128, 8), (16, 256, 32, 64, 2), (64, 128, 16, 32, 4),
+    (32, 512, 64, 128, 2), (64, 512, 64, 128, 8), (48, 512, 64, 128, 2),
 ])
 def test_ragged_batch(kernel, H, L, R, dv, g):
     d = _case(len(RAGGED), H, L, R, dv, g, RAGGED, seed=3 + H + g)
