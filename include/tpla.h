@@ -24,6 +24,16 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work
  *     is enqueued asynchronously on it; nothing is synchronised unless the
  *     function says so.
+ *   - Kernels are launched with programmatic stream serialisation: one may
+ *     start while the previous kernel on the stream is finishing, if that
+ *     kernel allows it early.  This library's kernels allow it only after
+ *     their own wait, and wait for the previous kernel before they read any
+ *     argument, with one exception: the combine stage (tpla_combine, and the
+ *     second stage of tpla_decode / tpla_decode_shard / mla_decode) reads
+ *     w_uv and seq_lens before that wait.  So when tpla_combine follows a
+ *     kernel of the caller's own that signals programmatic completion early
+ *     (griddepcontrol.launch_dependents), that kernel must not write w_uv or
+ *     seq_lens after its signal.
  *   - Return value: TPLA_OK, or a tpla_status_t.  A non-zero status means
  *     nothing was enqueued, except TPLA_ERR_CUDA (a launch failed).
  *     Errors that only the device can see (a sequence longer than its
