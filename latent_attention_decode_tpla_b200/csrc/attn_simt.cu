@@ -7,9 +7,11 @@
 //     o_{h,s} = sum_t softmax(z)_t c_{t,s}
 // computed as an online (streaming) softmax over 64-token tiles, one split-KV
 // segment at a time (schedule in tpla_internal.cuh).  This kernel uses plain
-// fp32 FMAs; it serves every supported shape and is the yardstick the
-// tcgen05 kernel is tested against.  One CTA = one worker x a group of 16
-// heads; every CTA of a worker walks the same units.
+// fp32 FMAs on register tiles; it serves every supported shape (it is the
+// path for g = 1, whose O does not fit in tensor memory beside S and the
+// query) and is the yardstick the tcgen05 kernel is tested against.  One
+// CTA = one worker x a group of 16 heads; every CTA of a worker walks the
+// same units.
 #include "tpla_internal.cuh"
 
 #include <cuda_bf16.h>
