@@ -22,7 +22,7 @@ Disaggregated Prefill & Decode Inference", arXiv 2508.15881):
   [PBOT]  paperbot summary page, extended abstract: the cache is named cKV;
           RMSNorm and softmax get orthogonal reparameterisations.
 
-Readings where the pages are silent (each is also listed in the design doc):
+Readings where the pages are silent:
   * the decoupled RoPE key is replicated: every shard adds the full
     q_pe . k_pe term to its scores;
   * the softmax scale is the caller's ``scale`` for every shard (no
