@@ -31,6 +31,7 @@ Readings where the pages are silent:
   * transform first, then per-shard RMSNorm: y = R x, c_s = y_s / sqrt(mean(y_s^2) + eps),
     optionally times a weight in the transformed basis;
   * Hadamard = Sylvester construction in natural order, scaled by 1/sqrt(L);
+    the block variant applies H_{L/g} / sqrt(L/g) to each shard's slice alone;
   * stored cache values are rounded to bfloat16, round-to-nearest-even;
   * tokens at positions >= seq_len are ignored; an empty sequence gives 0.
 
@@ -45,6 +46,7 @@ PAGE_SIZE = 64          # tokens per cache page (layout of the paged latent cach
 TRANSFORM_NONE = 0
 TRANSFORM_HADAMARD = 1
 TRANSFORM_DENSE = 2
+TRANSFORM_BLOCK_HADAMARD = 3
 
 
 # --------------------------------------------------------------------------
@@ -86,16 +88,29 @@ def sylvester_hadamard(n):
     return h
 
 
-def transform_matrix(transform, L, R_dense=None):
+def transform_matrix(transform, L, R_dense=None, g=1):
     """The L x L orthogonal matrix R applied to each new latent before slicing.
 
     transform 0: identity; 1: Sylvester Hadamard / sqrt(L); 2: the caller's dense
-    matrix (the PCA stand-in; a seeded random orthogonal matrix in the tests).
+    matrix (the PCA stand-in; a seeded random orthogonal matrix in the tests);
+    3: block-diagonal, one Sylvester Hadamard / sqrt(L/g) per shard slice of
+    L/g columns, so that each shard's values come from its own slice of the raw
+    latent only (a "Hadamard-like" transform cheaper than the full one, the
+    pages' named direction for future transforms; the full transform is the
+    g = 1 case).
     """
     if transform == TRANSFORM_NONE:
         return np.eye(L)
     if transform == TRANSFORM_HADAMARD:
         return sylvester_hadamard(L) / np.sqrt(L)
+    if transform == TRANSFORM_BLOCK_HADAMARD:
+        if L % g:
+            raise ValueError("L must be divisible by g")
+        Ls = L // g
+        m = np.zeros((L, L))
+        for s in range(g):
+            m[s * Ls:(s + 1) * Ls, s * Ls:(s + 1) * Ls] = sylvester_hadamard(Ls) / np.sqrt(Ls)
+        return m
     if transform == TRANSFORM_DENSE:
         if R_dense is None:
             raise ValueError("dense transform needs R_dense")
@@ -117,7 +132,7 @@ def append_values(latent_raw, g, transform=TRANSFORM_HADAMARD, R_dense=None,
     if L % g:
         raise ValueError("L must be divisible by g")
     Ls = L // g
-    Rm = transform_matrix(transform, L, R_dense)
+    Rm = transform_matrix(transform, L, R_dense, g)
     y = x @ Rm.T                                    # y_b = R x_b
     ys = y.reshape(B, g, Ls)
     ms = np.mean(ys * ys, axis=2, keepdims=True)

@@ -81,6 +81,39 @@ def test_dense_transform_is_caller_matrix_and_orthogonal():
     np.testing.assert_allclose(t @ t.T, np.eye(64), atol=1e-6)
 
 
+@pytest.mark.parametrize("L,g", [(4, 2), (64, 4), (512, 2), (512, 8)])
+def test_block_hadamard_is_per_shard_sylvester(L, g):
+    # library routine: scipy's Sylvester Hadamard of order L/g on every diagonal block, zero elsewhere
+    Ls = L // g
+    t = ref.transform_matrix(ref.TRANSFORM_BLOCK_HADAMARD, L, None, g)
+    want = scipy.linalg.block_diag(*([scipy.linalg.hadamard(Ls) / math.sqrt(Ls)] * g))
+    np.testing.assert_allclose(t, want, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(t @ t.T, np.eye(L), atol=1e-13)
+    # one block is the full transform
+    np.testing.assert_array_equal(ref.transform_matrix(ref.TRANSFORM_BLOCK_HADAMARD, L, None, 1),
+                                  ref.transform_matrix(ref.TRANSFORM_HADAMARD, L))
+
+
+def test_block_hadamard_append_hand_worked_and_shard_local():
+    # L = 4, g = 2: each shard's pair (a, b) becomes ((a + b), (a - b)) / sqrt(2), then its own RMSNorm.
+    # x = [3, 1, 2, -2]: shard 0 -> [4, 2] / sqrt 2, mean square 5, so c_0 = [4, 2] / sqrt(2 (5 + eps));
+    # shard 1 -> [0, 4] / sqrt 2, mean square 4, so c_1 = [0, 4] / sqrt(2 (4 + eps)).
+    eps = 1e-6
+    c = ref.append_values(np.array([[3.0, 1.0, 2.0, -2.0]]), 2, ref.TRANSFORM_BLOCK_HADAMARD, None, None, eps)
+    np.testing.assert_allclose(c[0, 0], np.array([4.0, 2.0]) / math.sqrt(2 * (5 + eps)), rtol=1e-15)
+    np.testing.assert_allclose(c[0, 1], np.array([0.0, 4.0]) / math.sqrt(2 * (4 + eps)), rtol=1e-15)
+    # the full transform mixes the shards: the same input gives other values
+    full = ref.append_values(np.array([[3.0, 1.0, 2.0, -2.0]]), 2, ref.TRANSFORM_HADAMARD, None, None, eps)
+    assert np.max(np.abs(full - c)) > 0.1
+    # a one-hot input in shard 2 of 4 leaves every other shard zero (no mixing across shards)
+    L, g = 64, 4
+    x = np.zeros((1, L)); x[0, 2 * 16 + 5] = 1.0
+    cb = ref.append_values(x, g, ref.TRANSFORM_BLOCK_HADAMARD, None, None, eps)
+    for s in range(g):
+        assert np.all(cb[0, s] == 0.0) == (s != 2)
+    np.testing.assert_allclose(cb[0, 2], scipy.linalg.hadamard(16)[:, 5] / math.sqrt(1 + 16 * eps), rtol=1e-14)
+
+
 # ---------------------------------------------------------------- append (transform + sliced RMSNorm)
 
 def test_append_g1_equals_transform_of_rmsnorm():
@@ -169,8 +202,11 @@ def _small_case(B, H, L, R, dv, g, lens, seed, shuffle=True, dn=None):
                 maxp=d["max_pages_per_seq"], raw=d)
 
 
-def _brute_force(c, scale, shard_only=None, latent=False):
-    """Scalar loops over b, h, s, t with an explicit page walk (no numpy algebra)."""
+def _brute_force(c, scale, shard_only=None, latent=False, probs=None):
+    """Scalar loops over b, h, s, t with an explicit page walk (no numpy algebra).
+
+    If ``probs`` is a dict, the softmax weights of every (b, s) with T_b > 0 are
+    stored in it as probs[(b, s)][h][t]."""
     q, q_pe, ckv, kpe, bt, lens, w = c["q"], c["q_pe"], c["ckv"], c["kpe"], c["bt"], c["lens"], c["w_uv"]
     B, H, L = q.shape
     g = ckv.shape[1]
@@ -197,6 +233,8 @@ def _brute_force(c, scale, shard_only=None, latent=False):
                 m = max(zs)
                 es = [math.exp(z - m) for z in zs]
                 den = sum(es)
+                if probs is not None:
+                    probs.setdefault((b, s), [None] * H)[h] = [e / den for e in es]
                 o = [0.0] * Ls
                 for t in range(T):
                     page, slot = bt[b][t // 64], t % 64
@@ -306,6 +344,27 @@ def test_shard_softmax_rows_sum_to_one():
             assert p.shape == (5, int(c["lens"][b]))
             assert np.all(p >= 0)
             np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+
+
+def test_shard_probabilities_match_brute_force():
+    # every (sequence, shard) of a g = 4 case on a shuffled page table, including a one-token
+    # sequence and tails that end inside a page: the weights must be the brute-force loop's
+    # exp(z - max) / sum, head by head and token by token
+    c = _small_case(B=3, H=3, L=32, R=4, dv=2, g=4, lens=[1, 70, 129], seed=43)
+    scale = 0.45
+    probs = {}
+    _brute_force(c, scale, probs=probs)
+    for b in range(3):
+        for s in range(4):
+            p = ref.shard_probabilities(c["q"], c["q_pe"], c["ckv"], c["kpe"], c["bt"], c["lens"], scale,
+                                        b, s, max_pages_per_seq=c["maxp"])
+            np.testing.assert_allclose(p, np.array(probs[(b, s)]), rtol=0, atol=1e-14)
+    # and the weights of different shards differ (each shard has its own softmax)
+    p0 = ref.shard_probabilities(c["q"], c["q_pe"], c["ckv"], c["kpe"], c["bt"], c["lens"], scale, 2, 0,
+                                 max_pages_per_seq=c["maxp"])
+    p3 = ref.shard_probabilities(c["q"], c["q_pe"], c["ckv"], c["kpe"], c["bt"], c["lens"], scale, 2, 3,
+                                 max_pages_per_seq=c["maxp"])
+    assert np.max(np.abs(p0 - p3)) > 1e-3
 
 
 def _to_g1(ckv):
