@@ -204,7 +204,8 @@ int tpla_decode_static(const tpla_dims_t* dims,
  * and sums over shards into `out`, exactly as tpla_decode /
  * tpla_decode_shard document.  The combine must use the same dims, shard,
  * seq_lens contents and workspace as the attention call before it, on the
- * same stream (or after it in stream order).
+ * same stream (or after it in stream order), with the same options set (the options decide the
+ * attention kernel, and with it the split-KV worker count the combine expects).
  */
 int tpla_attention(const tpla_dims_t* dims, int shard,
                    const tpla_bf16* q_nope_absorbed, const tpla_bf16* q_pe,
@@ -220,6 +221,11 @@ int tpla_combine(const tpla_dims_t* dims, int shard, const int32_t* seq_lens,
 #define TPLA_TRANSFORM_NONE      0   /* identity */
 #define TPLA_TRANSFORM_HADAMARD  1   /* Sylvester Hadamard / sqrt(L), natural order; L a power of two */
 #define TPLA_TRANSFORM_DENSE     2   /* caller's orthogonal R_dense (e.g. a PCA basis) */
+#define TPLA_TRANSFORM_BLOCK_HADAMARD 3  /* block-diagonal: Sylvester Hadamard / sqrt(L/g) on each
+                                            shard's L/g columns of x, so a shard's values depend on
+                                            its own slice only (edgentiq blog, "Real-World Impact
+                                            and Future Directions": cheaper Hadamard-like transforms
+                                            as the next step); equals HADAMARD when g == 1 */
 
 /*
  * tpla_append_kv -- write one new token per sequence into the cache
@@ -231,7 +237,8 @@ int tpla_combine(const tpla_dims_t* dims, int shard, const int32_t* seq_lens,
  * with page = block_table[b][positions[b] / 64] (or the identity layout) and
  * slot = positions[b] % 64.
  *   latent_raw  [B][L] bf16;  kpe_new [B][R] bf16 (post-RoPE);
- *   transform   TPLA_TRANSFORM_*;  R_dense [L][L] fp32 row-major (y_i = sum_j R[i][j] x_j),
+ *   transform   TPLA_TRANSFORM_* (an unknown value returns TPLA_ERR_INVALID_ARG);
+ *               R_dense [L][L] fp32 row-major (y_i = sum_j R[i][j] x_j),
  *               required for TPLA_TRANSFORM_DENSE, ignored otherwise;
  *   norm_weight [L] fp32 or NULL (weight applied in the transformed basis);
  *   eps         added to the mean square (>= 0);
@@ -255,13 +262,16 @@ int tpla_append_kv(const tpla_dims_t* dims,
 int tpla_check_device_status(void* stream);
 
 /* Options (process-wide, for testing and tuning). */
-#define TPLA_OPT_ATTENTION_KERNEL  1  /* 0 auto (tcgen05 where supported), 1 CUDA-core kernel, 2 tcgen05 kernel */
+#define TPLA_OPT_ATTENTION_KERNEL  1  /* 0 auto (tcgen05 where supported), 1 CUDA-core kernel, 2 tcgen05 kernel
+                                         (R == 64 and L/g in {64, 128, 256, 512}; other shapes return
+                                         TPLA_ERR_UNSUPPORTED) */
 #define TPLA_OPT_MAX_WORKERS       2  /* cap on split-KV workers per call (0 = one per SM) */
 #define TPLA_OPT_WAIT_LIMIT        3  /* spin iterations before a pipeline wait gives up (0 = default) */
 #define TPLA_OPT_DEBUG_STALL       4  /* 1: the tcgen05 kernel waits on a barrier nothing signals, to
                                          exercise the bounded-wait path (returns TPLA_ERR_TIMEOUT) */
 #define TPLA_OPT_LAST_ATTENTION_KERNEL 5  /* read-only: kernel of the last attention launch in this
-                                             process (0 none yet, 1 CUDA-core, 2 tcgen05) */
+                                             process (0 none yet, 1 CUDA-core, 2 tcgen05 with 128-token
+                                             tiles (L/g <= 256), 3 tcgen05 CTA pair (L/g == 512)) */
 int tpla_set_option(int option, int value);
 int tpla_get_option(int option);
 

@@ -122,10 +122,17 @@ int make_plan(const tpla_dims_t* d, int shard, Plan* p) {
     p->num_pages = d->num_pages;
     p->scale_log2 = d->softmax_scale * kLog2e;
     p->status = status;
-    int cap = sms < kMaxWorkers ? sms : kMaxWorkers;
+    // the attention kernel: tcgen05 where the shape has a variant (unless the CUDA-core kernel is
+    // forced), else the CUDA-core kernel; a forced tcgen05 kernel without a variant is an error
+    const bool tc = sm100_supports(*p), wide = sm100_wide_supports(*p);
+    if (g_opt_kernel == 2 && !tc && !wide) return TPLA_ERR_UNSUPPORTED;
+    p->kernel = g_opt_kernel == 1 ? kKernelSimt : (tc ? kKernelSm100 : (wide ? kKernelSm100Wide : kKernelSimt));
+    // workers: one per SM (a CTA pair per worker for the wide kernel), at most kMaxWorkers
+    int cap = p->kernel == kKernelSm100Wide ? sms / 2 : sms;
+    cap = cap < kMaxWorkers ? cap : kMaxWorkers;
     if (g_opt_max_workers > 0 && g_opt_max_workers < cap) cap = g_opt_max_workers;
     const long long umax = (long long)p->gc * d->B * d->max_pages_per_seq;
-    const int min_units = sm100_supports(*p) ? kMinUnitsPerWorker : 1;
+    const int min_units = p->kernel == kKernelSm100 ? kMinUnitsPerWorker : 1;
     long long w = (umax + min_units - 1) / min_units;
     w = w < 1 ? 1 : (w > cap ? cap : w);
     // With a multiple of the (sequence, shard) pair count as the worker count, equal-length pairs
@@ -140,13 +147,44 @@ int make_plan(const tpla_dims_t* d, int shard, Plan* p) {
     return TPLA_OK;
 }
 
-Workspace carve(void* workspace, const tpla_dims_t* d, size_t slots = 0) {
-    if (slots == 0) slots = (size_t)kMaxWorkers + (size_t)d->B * d->g;
+// Workspace: 256-byte header | log-sum-exps | partial outputs.  The log-sum-exp block is sized for
+// kMaxWorkers + B*g slots in every path (ws_lse_bytes), so the partial outputs start at the same
+// offset whatever worker count a call uses; the partial region needs (W + B*g) slots of H*(L/g)
+// floats, which the caller's workspace (sized for kMaxWorkers) and the static scratch (W clamped
+// to fit) both provide.
+Workspace carve(void* workspace, const tpla_dims_t* d) {
     char* base = static_cast<char*>(workspace) + 256;
     Workspace w;
     w.part_lse = reinterpret_cast<float*>(base);
     w.part_o = reinterpret_cast<float*>(base + ws_lse_bytes(d));
     return w;
+}
+
+// The attention pass of plan p, on the kernel the plan chose; records which one was launched.
+int launch_attention(const Plan& p, const tpla_bf16* q, const tpla_bf16* q_pe, const tpla_bf16* ckv,
+                     const tpla_bf16* kpe, const int32_t* block_table, const int32_t* seq_lens, Workspace w,
+                     cudaStream_t s) {
+    auto bq = reinterpret_cast<const __nv_bfloat16*>(q);
+    auto bqp = reinterpret_cast<const __nv_bfloat16*>(q_pe);
+    auto bc = reinterpret_cast<const __nv_bfloat16*>(ckv);
+    auto bk = reinterpret_cast<const __nv_bfloat16*>(kpe);
+    cudaError_t e;
+    switch (p.kernel) {
+        case kKernelSm100:
+            e = launch_attention_sm100(p, bq, bqp, bc, bk, block_table, seq_lens, w, g_opt_wait_limit,
+                                       g_opt_debug_stall, s);
+            break;
+        case kKernelSm100Wide:
+            e = launch_attention_sm100_wide(p, bq, bqp, bc, bk, block_table, seq_lens, w, g_opt_wait_limit,
+                                            g_opt_debug_stall, s);
+            break;
+        default:
+            e = launch_attention_simt(p, bq, bqp, bc, bk, block_table, seq_lens, w, s);
+            break;
+    }
+    g_last_kernel = p.kernel;
+    if (e == cudaErrorNotSupported) return TPLA_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? TPLA_OK : TPLA_ERR_CUDA;
 }
 
 int run_attention(const tpla_dims_t* d, int shard, const tpla_bf16* q, const tpla_bf16* q_pe,
@@ -156,25 +194,8 @@ int run_attention(const tpla_dims_t* d, int shard, const tpla_bf16* q, const tpl
     if (st || d->B == 0) return st;
     Plan p;
     if ((st = make_plan(d, shard, &p))) return st;
-    Workspace w = carve(workspace, d);
-    auto bq = reinterpret_cast<const __nv_bfloat16*>(q);
-    auto bqp = reinterpret_cast<const __nv_bfloat16*>(q_pe);
-    auto bc = reinterpret_cast<const __nv_bfloat16*>(ckv);
-    auto bk = reinterpret_cast<const __nv_bfloat16*>(kpe);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    const bool tc_ok = sm100_supports(p);
-    if (g_opt_kernel == 2 && !tc_ok) return TPLA_ERR_UNSUPPORTED;
-    if (g_opt_kernel != 1 && tc_ok) {
-        e = launch_attention_sm100(p, bq, bqp, bc, bk, block_table, seq_lens, w, g_opt_wait_limit,
-                                   g_opt_debug_stall, s);
-        g_last_kernel = 2;
-    } else {
-        e = launch_attention_simt(p, bq, bqp, bc, bk, block_table, seq_lens, w, s);
-        g_last_kernel = 1;
-    }
-    if (e == cudaErrorNotSupported) return TPLA_ERR_UNSUPPORTED;
-    return e == cudaSuccess ? TPLA_OK : TPLA_ERR_CUDA;
+    return launch_attention(p, q, q_pe, ckv, kpe, block_table, seq_lens, carve(workspace, d),
+                            static_cast<cudaStream_t>(stream));
 }
 
 int run_combine(const tpla_dims_t* d, int shard, const int32_t* seq_lens, const tpla_bf16* w_uv,
@@ -277,7 +298,7 @@ int tpla_append_kv(const tpla_dims_t* dims, const tpla_bf16* latent_raw, const t
                    tpla_bf16* kpe_cache, void* stream) {
     int st = check_dims(dims);
     if (st) return st;
-    if (transform < TPLA_TRANSFORM_NONE || transform > TPLA_TRANSFORM_DENSE) return TPLA_ERR_INVALID_ARG;
+    if (transform < TPLA_TRANSFORM_NONE || transform > TPLA_TRANSFORM_BLOCK_HADAMARD) return TPLA_ERR_INVALID_ARG;
     if (!(eps >= 0.f) || !std::isfinite(eps)) return TPLA_ERR_INVALID_ARG;
     if (dims->B == 0) return TPLA_OK;
     if (!latent_raw || !kpe_new || !positions || !ckv_cache || !kpe_cache) return TPLA_ERR_INVALID_ARG;
@@ -407,18 +428,10 @@ extern "C" int tpla_decode_static(const tpla_dims_t* dims, const tpla_bf16* q, c
     Plan p;
     if ((st = make_plan(dims, -1, &p))) return st;
     if (p.W > max_slots - fixed) p.W = (int)(max_slots - fixed);  // fewer split-KV workers, same result
-    Workspace w = carve(scratch, dims, (size_t)p.W + (size_t)fixed);
+    // (W + B*g) partial slots follow the log-sum-exp block, which carve() sizes for kMaxWorkers + B*g
+    Workspace w = carve(scratch, dims);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    auto bq = reinterpret_cast<const __nv_bfloat16*>(q);
-    auto bqp = reinterpret_cast<const __nv_bfloat16*>(q_pe);
-    auto bc = reinterpret_cast<const __nv_bfloat16*>(ckv);
-    auto bk = reinterpret_cast<const __nv_bfloat16*>(kpe);
-    cudaError_t e = sm100_supports(p) && g_opt_kernel != 1
-                        ? launch_attention_sm100(p, bq, bqp, bc, bk, block_table, seq_lens, w, g_opt_wait_limit,
-                                                 g_opt_debug_stall, s)
-                        : launch_attention_simt(p, bq, bqp, bc, bk, block_table, seq_lens, w, s);
-    if (e == cudaErrorNotSupported) return TPLA_ERR_UNSUPPORTED;
-    if (e != cudaSuccess) return TPLA_ERR_CUDA;
-    e = launch_combine(p, seq_lens, reinterpret_cast<const __nv_bfloat16*>(w_uv), out, w, s);
+    if ((st = launch_attention(p, q, q_pe, ckv, kpe, block_table, seq_lens, w, s))) return st;
+    cudaError_t e = launch_combine(p, seq_lens, reinterpret_cast<const __nv_bfloat16*>(w_uv), out, w, s);
     return e == cudaSuccess ? TPLA_OK : TPLA_ERR_CUDA;
 }

@@ -4,7 +4,9 @@
 // an orthogonal transform (Hadamard or PCA) is applied to the latent before
 // it is cut into shards, so that the RMSNorm each shard computes on its own
 // slice stays close to the global one.  Per new token b:
-//     y   = R x_b                      (Hadamard: fast Walsh-Hadamard transform, 1/sqrt(L))
+//     y   = R x_b                      (Hadamard: fast Walsh-Hadamard transform, 1/sqrt(L);
+//                                       block Hadamard: the same butterflies restricted to each
+//                                       shard's L/g columns, 1/sqrt(L/g))
 //     c_s = y_s / sqrt(mean(y_s^2) + eps)  [* w_s]   for every shard s
 // rounded to bf16 (round to nearest even) and written to
 // ckv[page][s][slot][:], with k_pe copied to kpe[page][slot][:].
@@ -52,29 +54,33 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
     }
     const int slot = pos % kPage;
 
+    // butterfly span: the whole latent, or one shard's slice for the block-diagonal transform
+    // (butterflies of stride h < L/g only pair indices of the same L/g-aligned block)
+    const bool hadamard = transform == TPLA_TRANSFORM_HADAMARD || transform == TPLA_TRANSFORM_BLOCK_HADAMARD;
+    const int hn = transform == TPLA_TRANSFORM_BLOCK_HADAMARD ? Ls : L;
     float xv = 0.f;                                   // x[tid] when L <= kThreads
     if (L <= kThreads) {
         if (tid < L) xv = __bfloat162float(latent_raw[(size_t)b * L + tid]);
-        if (transform != TPLA_TRANSFORM_HADAMARD && tid < L) x[tid] = xv;
+        if (!hadamard && tid < L) x[tid] = xv;
     } else {
         for (int i = tid; i < L; i += kThreads) x[i] = __bfloat162float(latent_raw[(size_t)b * L + i]);
     }
     __syncthreads();
 
-    if (transform == TPLA_TRANSFORM_HADAMARD && L <= kThreads) {
-        // Radix-2 butterflies over L = 2^k points (Sylvester order), one point per thread: the
+    if (hadamard && L <= kThreads) {
+        // Radix-2 butterflies over hn = 2^k points (Sylvester order), one point per thread: the
         // pair (i, i + h) of stage h becomes (a + c, a - c).  Strides below 32 pair lanes of one
         // warp (shuffles); wider strides go through shared memory, alternating two buffers so
         // that one barrier per stage suffices.  Whole warps are idle when tid >= L (L >= 64).
         float v = xv;
         if (tid < L) {
-            for (int h = 1; h < 32 && h < L; h <<= 1) {
+            for (int h = 1; h < 32 && h < hn; h <<= 1) {
                 const float o = __shfl_xor_sync(0xffffffffu, v, h);
                 v = (tid & h) ? o - v : v + o;
             }
         }
         int buf = 0;
-        for (int h = 32; h < L; h <<= 1) {
+        for (int h = 32; h < hn; h <<= 1) {
             float* yb = buf ? y : x;
             if (tid < L) yb[tid] = v;
             __syncthreads();
@@ -85,12 +91,12 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
             buf ^= 1;
         }
         __syncthreads();   // every read of the last stage's buffer is done before y is written
-        if (tid < L) y[tid] = v * (1.0f / sqrtf((float)L));
-    } else if (transform == TPLA_TRANSFORM_HADAMARD) {
-        // in-place radix-2 butterflies over L = 2^k points (Sylvester order), then 1/sqrt(L)
+        if (tid < L) y[tid] = v * (1.0f / sqrtf((float)hn));
+    } else if (hadamard) {
+        // in-place radix-2 butterflies of stride < hn (Sylvester order), then 1/sqrt(hn)
         for (int i = tid; i < L; i += kThreads) y[i] = x[i];
         __syncthreads();
-        for (int hlen = 1; hlen < L; hlen <<= 1) {
+        for (int hlen = 1; hlen < hn; hlen <<= 1) {
             for (int k = tid; k < L / 2; k += kThreads) {
                 int i = (k / hlen) * 2 * hlen + (k % hlen);
                 float a = y[i], c = y[i + hlen];
@@ -99,7 +105,7 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
             }
             __syncthreads();
         }
-        const float sc = 1.0f / sqrtf((float)L);
+        const float sc = 1.0f / sqrtf((float)hn);
         for (int i = tid; i < L; i += kThreads) y[i] *= sc;
     } else if (transform == TPLA_TRANSFORM_DENSE) {
         // y_i = sum_j R[i][j] x_j for the shard's rows: each warp takes four rows at a time,

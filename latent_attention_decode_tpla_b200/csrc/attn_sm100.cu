@@ -35,14 +35,19 @@
 // bf16 (8 significant bits) gives outputs with about 1.2e-3 relative RMS
 // error on sequences of a few hundred tokens, falling to 3-7e-4 at 4K-32K
 // tokens (the output's systematic part grows with length while the rounding
-// noise averages out).  So a segment of a sequence shorter than
-// kExactPVBelow tokens runs PV in fp16 (11 bits, about 1.5e-4): one MMA never
+// noise averages out).  So the tiles of a sequence shorter than
+// kExactPVBelow tokens run PV in fp16 (11 bits, about 1.5e-4): one MMA never
 // mixes the two types, so after QK^T of such a tile has completed the softmax
-// warps convert its latent rows in shared memory from bf16 to fp16 in place
-// (each bf16 value of the RMS-normalised cache is exactly an fp16 value
-// unless its magnitude is below 2^-14).  Longer sequences keep the bf16 tile
-// and bf16 P, which costs no extra shared-memory traffic.  In both modes the
-// rows past the end of the sequence are zeroed before PV reads the tile.
+// warps convert its latent rows in shared memory from bf16 to fp16 in place.
+// A bf16 value is exactly an fp16 value only between 2^-14 and 65504, and the
+// cache is the caller's (any transform, any norm weight), so each such tile
+// first takes the maximum |value| of its valid rows across the softmax warps
+// and scales the tile by a power of two (and P by its inverse) to bring that
+// maximum into fp16's range, keeping bf16 only for tiles beyond that
+// (pv_fp16_shift in attn_sm100_common.cuh).
+// Longer sequences keep the bf16 tile and bf16 P, which costs no extra
+// shared-memory traffic.  In both modes the rows past the end of the sequence
+// are zeroed before PV reads the tile.
 // All exponentials run on the special-function unit: moving a share of them
 // to a polynomial on the FMA pipe measured slower here, since the softmax is
 // bound by its latency chain, not by that unit's throughput.
@@ -65,9 +70,7 @@
 // barrier while another may have stopped.
 #include "tpla_internal.cuh"
 #include "sm100_ptx.cuh"
-
-#include <cuda.h>
-#include <mutex>
+#include "attn_sm100_common.cuh"
 
 namespace tpla {
 namespace {
@@ -112,75 +115,14 @@ struct Bars {
     uint64_t full[NST];
     uint64_t empty[NST];
     uint64_t s_full, s_free, p_full, o_done;
-    uint64_t q_full, o_free, xmax, xsum, drain, never;
+    uint64_t q_full, o_free, xmax, xsum, drain, never, vote;
     float xmax_buf[2][2][128];     // [tile parity][warpgroup][row]
     float xsum_buf[2][2][128];     // [segment parity][warpgroup][row]
+    uint32_t vote_max[2][8];       // [tile parity][softmax warp]: largest |latent| bit pattern seen
+    int pv_f16[2];                 // [tile parity]: PV of that tile runs in fp16
     uint32_t tmem_base;
     volatile int abort;
 };
-
-struct Waiter {
-    volatile int* abort;
-    unsigned* status;
-    uint64_t limit_cycles;
-
-    // true when the phase of `parity` completed; false on abort or time-out
-    // (the limit is counted in SM clock cycles: reading %globaltimer in the loop is slow)
-    __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
-        if (mbar_try_wait(bar, parity)) return true;
-        const long long t0 = clock64();
-        for (;;) {
-            if (mbar_try_wait(bar, parity)) return true;
-            if (*abort) return false;
-            if ((uint64_t)(clock64() - t0) > limit_cycles) {
-                atomicOr(status, kStatusTimeout);
-                *abort = 1;
-                return false;
-            }
-        }
-    }
-};
-
-// A tile: one or two consecutive units (pages) of one (sequence, shard) segment.
-struct Tile {
-    UnitPos pos;      // first unit of the tile
-    long long u;      // its index in the unit order
-    int npages;       // 1 or 2
-    bool begin, end;  // first / last tile of its segment
-};
-
-__device__ __forceinline__ Tile make_tile(const UnitPos& pos, long long u, long long lo, long long hi) {
-    Tile t;
-    t.pos = pos;
-    t.u = u;
-    const long long left_seg = pos.ntiles - pos.tile;   // pages of this (b, s) from u on
-    const long long left_rng = hi - u;                 // units of the worker from u on
-    const long long left = left_seg < left_rng ? left_seg : left_rng;
-    t.npages = left >= 2 ? 2 : 1;
-    t.begin = u == lo || pos.tile == 0;
-    t.end = t.npages == left;
-    return t;
-}
-
-// the tile after `t`
-__device__ __forceinline__ Tile next_tile(const Tile& t, const int32_t* seq_lens, const Plan& p, long long lo,
-                                          long long hi) {
-    UnitPos pos = t.pos;
-    advance_unit(pos, seq_lens, p.B, p.max_pages, p.gc);
-    if (t.npages == 2) advance_unit(pos, seq_lens, p.B, p.max_pages, p.gc);
-    return make_tile(pos, t.u + t.npages, lo, hi);
-}
-
-// warp-collective: all lanes of the warp arrive through lane 0 after their prior writes
-__device__ __forceinline__ void warp_arrive(uint32_t bar) {
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
-// byte offset of 16-byte piece `c` of row `r` in a 128B-swizzled K-major operand (rows of 128 bytes)
-__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
-    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
-}
 
 template <int LS, int RD, int NST, bool HALF>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -220,6 +162,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         mbar_init(smem_addr(&bars.xsum), kSoftmaxWarps);
         mbar_init(smem_addr(&bars.drain), 1);
         mbar_init(smem_addr(&bars.never), 1);
+        mbar_init(smem_addr(&bars.vote), kSoftmaxWarps);
         bars.abort = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -292,7 +235,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 }
                 return page;
             };
-            Tile t = make_tile(pos0, lo, lo, hi);
+            Tile t = make_tile(pos0, lo, lo, hi, 2);
             long long j = 0;
             for (; t.u < hi; ++j) {
                 const int st = (int)(j % NST);
@@ -353,17 +296,16 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             // for the next load.  (Issuing QK^T in several groups, to let a PV that becomes ready
             // meanwhile in sooner, measured much slower on B200: the issue of a group costs far
             // more than its MMAs.)  Each stream has its own tile cursor.
-            Tile tq = make_tile(pos0, lo, lo, hi), tv = tq;
+            Tile tq = make_tile(pos0, lo, lo, hi, 2), tv = tq;
             long long jq = 0, jv = 0;
             int qseg = -1, vseg = -1;
-            bool vbegun = false, vexact = false;
+            bool vbegun = false;
             long long idle_since = clock64();
             while (ok && tv.u < hi) {
                 bool did = false;
                 if (jv < jq) {
                     if (tv.begin && !vbegun) {
                         ++vseg;
-                        vexact = tv.pos.T < kExactPVBelow;
                         vbegun = true;
                     }
                     if (mbar_test_wait(smem_addr(&bars.p_full), (uint32_t)(jv & 1)) &&
@@ -372,13 +314,14 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                         tc_fence_after();
                         const int st = (int)(jv % NST);
                         const uint32_t sb = stage0 + st * C::kStageBytes;
+                        // the softmax warps chose this tile's PV type before they signalled P
+                        const uint32_t idesc_pv = bars.pv_f16[jv & 1] ? C::kIdescPVf16 : C::kIdescPVbf16;
 #pragma unroll
                         for (int kk = 0; kk < kTileTok / 16; ++kk) {
                             // A: 16 tokens of P (K-major); B: the same 16 token rows of every latent chunk (MN-major)
                             const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * C::kPChunk + (kk & 3) * 32, 16, 1024);
                             const uint64_t bd = smem_desc_sw128(sb + kk * 2048, C::kChunk, 1024);
-                            mma_ss(tmem + C::kColO, ad, bd, vexact ? C::kIdescPVf16 : C::kIdescPVbf16,
-                                   (tv.begin && kk == 0) ? 0u : 1u);
+                            mma_ss(tmem + C::kColO, ad, bd, idesc_pv, (tv.begin && kk == 0) ? 0u : 1u);
                         }
                         mma_commit(smem_addr(&bars.empty[st]));
                         mma_commit(smem_addr(&bars.o_done));
@@ -464,7 +407,8 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
         int seg = -1;
         float m = -INFINITY, l = 0.f;                     // l: this thread's part of the row sum
         bool first_tile = true;
-        bool exact = false;                               // fp16 PV for this segment
+        bool exact = false;                               // segment short enough for fp16 PV tiles
+        long long nvote = 0;                              // range votes taken (tiles of short segments)
         // PV(t) is the t-th completion of o_done; completions are in order, so observing PV(t)
         // covers all before it
         auto wait_o = [&](long long t) -> bool {
@@ -531,7 +475,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             for (int k = 0; k < 8; ++k)
                 *reinterpret_cast<uint4*>(p_smem + wg * C::kPChunk + sw128_offset(row, k)) = make_uint4(0, 0, 0, 0);
         }
-        Tile t = make_tile(pos0, lo, lo, hi);
+        Tile t = make_tile(pos0, lo, lo, hi, 2);
         load_q(pos0);
         long long j = 0;
         for (; t.u < hi; ++j) {
@@ -592,12 +536,37 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             const float m_ref = raise ? m_loc : (m > -INFINITY ? m : 0.f);  // 0: no valid column yet, P = 0
             bars.xmax_buf[j & 1][wg][row] = raise ? m_loc : -INFINITY;
             warp_arrive(smem_addr(&bars.xmax));
+            // PV type of this tile (pv_fp16_shift): a tile of a short segment, where the rounding of
+            // P would dominate the error, runs PV in fp16 with the latent values scaled by 2^e and P
+            // by 2^-e; from kExactPVBelow tokens on, and for tiles whose largest |value| is outside
+            // fp16's reach even when scaled, it keeps bf16.  The softmax warps agree on the tile's
+            // largest |value| through the vote barrier: each posts the largest bit pattern of |value|
+            // over its share of the tile's valid rows.
+            bool f16 = false;
+            float cshift = 1.f, pshift = 1.f;             // 2^e for the latent tile, 2^-e for P
+            if (exact) {
+                uint32_t mx = 0;
+#pragma unroll 4
+                for (int k = 0; k < C::kCvt; ++k) {
+                    const int i = tid_sm + k * kSoftmaxWarps * 32;
+                    const int rr = (i >> 3) & (kTileTok - 1);
+                    if (rr < valid) {
+                        const uint4 v =
+                            *reinterpret_cast<const uint4*>(sb + (i >> 10) * C::kChunk + rr * 128 + (i & 7) * 16);
+                        mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                                  __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
+                    }
+                }
+                mx = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
+                if (lane == 0) bars.vote_max[nvote & 1][sw] = mx;
+                warp_arrive(smem_addr(&bars.vote));
+            }
             uint32_t pk[kCols / 2];
             float lt = 0.f;
             auto pack = [&]() {
-                if (exact) {
+                if (f16) {
 #pragma unroll
-                    for (int k = 0; k < kCols / 2; ++k) pk[k] = pack_f16x2(s[2 * k], s[2 * k + 1]);
+                    for (int k = 0; k < kCols / 2; ++k) pk[k] = pack_f16x2(s[2 * k] * pshift, s[2 * k + 1] * pshift);
                 } else {
 #pragma unroll
                     for (int k = 0; k < kCols / 2; ++k) pk[k] = pack_bf16x2(s[2 * k], s[2 * k + 1]);
@@ -615,12 +584,25 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
 #pragma unroll
                 for (int k = 0; k < kCols; ++k) l4[k & 3] += s[k];
                 lt = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            }
+            if (exact) {
+                if (!wt.wait(smem_addr(&bars.vote), (uint32_t)(nvote & 1))) break;
+                uint32_t tmax = 0;
+#pragma unroll
+                for (int k = 0; k < kSoftmaxWarps; ++k) tmax = max(tmax, bars.vote_max[nvote & 1][k]);
+                ++nvote;
+                int e = 0;
+                f16 = pv_fp16_shift(tmax, e);
+                cshift = __int_as_float((127 + e) << 23);
+                pshift = __int_as_float((127 - e) << 23);
+            }
+            if (warp_active) {
                 pack();
             } else {
 #pragma unroll
                 for (int k = 0; k < kCols / 2; ++k) pk[k] = 0u;
             }
-            if (exact) {
+            if (f16) {
                 // this tile's latent rows -> fp16 (rows past the sequence end -> 0) for PV;
                 // QK^T has finished reading them.  The 128B swizzle only permutes the 16-byte
                 // pieces within a row, so row rr is the 128 bytes at rr * 128 of its chunk.
@@ -631,10 +613,10 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                     uint4* ptr = reinterpret_cast<uint4*>(sb + (i >> 10) * C::kChunk + rr * 128 + (i & 7) * 16);
                     uint4 v = *ptr;
                     if (rr < valid) {
-                        v.x = bf16x2_to_f16x2(v.x);
-                        v.y = bf16x2_to_f16x2(v.y);
-                        v.z = bf16x2_to_f16x2(v.z);
-                        v.w = bf16x2_to_f16x2(v.w);
+                        v.x = bf16x2_to_f16x2_scaled(v.x, cshift);
+                        v.y = bf16x2_to_f16x2_scaled(v.y, cshift);
+                        v.z = bf16x2_to_f16x2_scaled(v.z, cshift);
+                        v.w = bf16x2_to_f16x2_scaled(v.w, cshift);
                     } else {
                         v = make_uint4(0, 0, 0, 0);
                     }
@@ -703,6 +685,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                     *reinterpret_cast<uint4*>(pb + sw128_offset(hrow, k0 + k)) =
                         make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
             }
+            if (tid_sm == 0) bars.pv_f16[j & 1] = f16 ? 1 : 0;   // read by the issuer after p_full
             fence_proxy_async_smem();
             warp_arrive(smem_addr(&bars.p_full));
             first_tile = false;
@@ -771,50 +754,6 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
 }
 
 // ------------------------------------------------------------------ host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    });
-    return fn;
-}
-
-// 3-D fp32 tensor map over the partial outputs [slots][H][Ls] with a 32 x 32 x 1 box (32 columns of
-// 32 rows of one slot) and 128-byte swizzle, for the TMA stores of the epilogue
-bool make_map_o(CUtensorMap* m, void* base, uint64_t ls, uint64_t h, uint64_t slots) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {ls, h, slots};
-    cuuint64_t strides[2] = {ls * 4, h * ls * 4};
-    cuuint32_t box[3] = {32, 32, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 2-D bf16 tensor map over [rows][cols] with a 64 x 64 box and 128-byte swizzle
-bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 64};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <int LS, int RD, int NST, bool HALF>
 cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16* q_pe, const __nv_bfloat16* ckv,

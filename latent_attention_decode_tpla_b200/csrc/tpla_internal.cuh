@@ -25,6 +25,11 @@ constexpr int kPage = 64;            // tokens per cache page and per attention 
 constexpr int kMaxWorkers = 160;     // workspace is sized for this many split-KV workers
 constexpr float kLog2e = 1.4426950408889634f;
 
+// attention kernels (values of TPLA_OPT_LAST_ATTENTION_KERNEL)
+constexpr int kKernelSimt = 1;       // CUDA cores, any supported shape
+constexpr int kKernelSm100 = 2;      // tcgen05, L/g in {64, 128, 256}
+constexpr int kKernelSm100Wide = 3;  // tcgen05, L/g = 512, a CTA pair per worker
+
 // device status bits (tpla_check_device_status)
 constexpr unsigned kStatusIndex = 1u;
 constexpr unsigned kStatusTimeout = 2u;
@@ -35,7 +40,8 @@ struct Plan {
     int gc;            // shards handled by this call (g, or 1 for a single-shard call)
     int shard0;        // first shard index of the call
     int max_pages, num_pages;
-    int W;             // split-KV workers
+    int W;             // split-KV workers (a worker of the wide tcgen05 kernel is a CTA pair)
+    int kernel;        // attention kernel: kKernelSimt, kKernelSm100 or kKernelSm100Wide
     float scale_log2;  // softmax_scale * log2(e)
     unsigned* status;  // device status word (kStatus* bits)
 };
@@ -217,6 +223,13 @@ cudaError_t launch_attention_sm100(const Plan& p, const __nv_bfloat16* q, const 
                                    const int32_t* block_table, const int32_t* seq_lens,
                                    Workspace ws, int wait_limit, int debug_stall, cudaStream_t stream);
 bool sm100_supports(const Plan& p);
+
+// Returns cudaErrorNotSupported when the shape is not L/g = 512 with R = 64.
+cudaError_t launch_attention_sm100_wide(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16* q_pe,
+                                        const __nv_bfloat16* ckv, const __nv_bfloat16* kpe,
+                                        const int32_t* block_table, const int32_t* seq_lens,
+                                        Workspace ws, int wait_limit, int debug_stall, cudaStream_t stream);
+bool sm100_wide_supports(const Plan& p);
 
 cudaError_t launch_combine(const Plan& p, const int32_t* seq_lens, const __nv_bfloat16* w_uv,
                            float* out, Workspace ws, cudaStream_t stream);

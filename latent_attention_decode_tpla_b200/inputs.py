@@ -133,6 +133,7 @@ WORKLOADS = {
                     stds=dict(q_std=1 / math.sqrt(64), qpe_std=1 / math.sqrt(16),
                               x_std=1 / math.sqrt(64), kpe_std=1 / math.sqrt(16))),
     "mla_g1_dsv3_b1_4k": dict(B=1, H=128, L=512, R=64, dv=128, g=1, T=4096, qk_nope=128, transform=1),
+    "mla_g1_dsv3_b8_32k": dict(B=8, H=128, L=512, R=64, dv=128, g=1, T=32768, qk_nope=128, transform=1),
     "tpla_g2_dsv3_b1_32k": dict(B=1, H=128, L=512, R=64, dv=128, g=2, T=32768, qk_nope=128, transform=1),
     "tpla_g2_dsv3_b16_32k": dict(B=16, H=128, L=512, R=64, dv=128, g=2, T=32768, qk_nope=128, transform=1),
     "tpla_g4_kimi_b8_32k": dict(B=8, H=64, L=512, R=64, dv=128, g=4, T=32768, qk_nope=128, transform=2),

@@ -26,6 +26,7 @@ TPLA_ERR_INDEX = 7
 TRANSFORM_NONE = 0
 TRANSFORM_HADAMARD = 1
 TRANSFORM_DENSE = 2
+TRANSFORM_BLOCK_HADAMARD = 3
 
 OPT_ATTENTION_KERNEL = 1
 OPT_MAX_WORKERS = 2

@@ -13,6 +13,9 @@ MAX_ABS = 2e-2
 REL_RMS = 1e-3
 
 KERNELS = {"simt": 1, "sm100": 2}
+# kernels reported by TPLA_OPT_LAST_ATTENTION_KERNEL for each forced choice: the tcgen05 choice runs
+# the 128-token-tile kernel (2) for L/g <= 256 and the CTA-pair kernel (3) for L/g = 512
+RAN = {"simt": (1,), "sm100": (2, 3)}
 
 
 def to64(t):
@@ -80,7 +83,7 @@ def run_gpu(d, scale, mode="full", shard=0, with_wuv=True, dev=None, block_table
     torch.cuda.synchronize()
     assert tpla.check_device_status() == tpla.TPLA_OK
     if kernel is not None:
-        assert used == KERNELS[kernel], "asked for %s, ran kernel %d" % (kernel, used)
+        assert used in RAN[kernel], "asked for %s, ran kernel %d" % (kernel, used)
     return to64(out)
 
 

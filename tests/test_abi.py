@@ -108,6 +108,8 @@ def test_append_validation():
     args = [FAKE[0], FAKE[1]]
     rest = [FAKE[4], None, FAKE[6], FAKE[7], None]
     assert L.tpla_append_kv(ctypes.byref(d), *args, 7, None, None, 1e-6, *rest) == tpla.TPLA_ERR_INVALID_ARG
+    assert L.tpla_append_kv(ctypes.byref(d), *args, 4, None, None, 1e-6, *rest) == tpla.TPLA_ERR_INVALID_ARG
+    assert L.tpla_append_kv(ctypes.byref(d), *args, -1, None, None, 1e-6, *rest) == tpla.TPLA_ERR_INVALID_ARG
     assert L.tpla_append_kv(ctypes.byref(d), *args, 2, None, None, 1e-6, *rest) == tpla.TPLA_ERR_INVALID_ARG
     assert L.tpla_append_kv(ctypes.byref(d), *args, 1, None, None, -1.0, *rest) == tpla.TPLA_ERR_INVALID_ARG
     assert L.tpla_append_kv(ctypes.byref(d), None, FAKE[1], 1, None, None, 1e-6, *rest) == \

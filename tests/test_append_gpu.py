@@ -61,6 +61,9 @@ def test_layout_bit_exact(g):
     (ref.TRANSFORM_DENSE, 4, 512, False), (ref.TRANSFORM_DENSE, 2, 256, True),
     (ref.TRANSFORM_HADAMARD, 2, 64, False), (ref.TRANSFORM_NONE, 1, 512, False),
     (ref.TRANSFORM_HADAMARD, 8, 1024, False),
+    (ref.TRANSFORM_BLOCK_HADAMARD, 2, 512, False), (ref.TRANSFORM_BLOCK_HADAMARD, 4, 512, True),
+    (ref.TRANSFORM_BLOCK_HADAMARD, 8, 1024, False), (ref.TRANSFORM_BLOCK_HADAMARD, 1, 512, False),
+    (ref.TRANSFORM_BLOCK_HADAMARD, 2, 64, False),
 ])
 def test_values_within_one_ulp(transform, g, L, weight):
     B, R, maxp = 64, 64, 2

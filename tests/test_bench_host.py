@@ -55,7 +55,39 @@ def test_profiled_traffic_needs_matching_sources(tmp_path, monkeypatch):
     assert bench.profiled_traffic("attn_sm100", "w") == 123.0
 
 
-def test_kernel_digest_covers_only_its_sources():
-    # the attention digest is computed from the files that decide one attention launch
-    assert set(bench.KERNEL_SOURCES["attn_sm100"]) == {"attn_sm100.cu", "sm100_ptx.cuh", "tpla_internal.cuh", "api.cu"}
-    assert bench.source_digest("attn_sm100") != bench.source_digest()
+def _included(csrc, name, seen):
+    # the file and every local header it includes, transitively
+    if name in seen or not os.path.exists(os.path.join(csrc, name)):
+        return seen
+    seen.add(name)
+    for ln in open(os.path.join(csrc, name)):
+        if ln.startswith('#include "') and not ln.startswith('#include "../'):
+            _included(csrc, ln.split('"')[1], seen)
+    return seen
+
+
+@pytest.mark.parametrize("kernel", ["attn_sm100", "attn_sm100_wide"])
+def test_kernel_digest_covers_only_its_sources(kernel):
+    # the attention digest is computed from the files that decide one attention launch: the
+    # kernel's file, every header it includes, and the host-side plan (api.cu)
+    csrc = os.path.join(ROOT, "latent_attention_decode_tpla_b200", "csrc")
+    want = _included(csrc, kernel + ".cu", set()) | {"api.cu"}
+    assert set(bench.KERNEL_SOURCES[kernel]) == want
+    assert bench.source_digest(kernel) != bench.source_digest()
+
+
+def test_cache_replicas_defeat_l2():
+    # a step that reads more than twice the L2 needs no replica; a smaller cache is rotated over an
+    # even number of replicas whose bytes together exceed twice the L2
+    assert bench.cache_replicas(335_544_320) == 1
+    for per_step in (21_000_000, 4_718_592, 100_663_296, 1):
+        n = bench.cache_replicas(per_step)
+        assert n % 2 == 0 and n * per_step > 2 * bench.L2_BYTES
+        assert (n - 2) * per_step <= 2 * bench.L2_BYTES          # not more than needed (+1 for evenness)
+    assert "rotated" in bench.l2_note(14, 21_000_000) and "no flush" in bench.l2_note(1, 335_544_320)
+
+
+def test_percentile_interpolates():
+    assert bench.percentile([3.0, 1.0, 2.0], 0.5) == 2.0
+    assert bench.percentile([1.0, 2.0, 3.0, 4.0, 5.0, 6.0, 7.0, 8.0, 9.0, 10.0], 0.9) == pytest.approx(9.1)
+    assert bench.percentile([5.0], 0.9) == 5.0

@@ -3,8 +3,7 @@
 Inputs are seeded and identical on both sides (bf16 values).  Tolerances on
 the fp32 outputs: max-abs <= 2e-2 and relative RMS <= 1e-3.  Small cases span
 several 64-token tiles, ragged tails and empty sequences; the benchmark
-configurations run at full size, with the oracle evaluated on a sample of
-sequences where the whole batch would take too long on the CPU.
+configurations run at full size, every sequence compared with the oracle.
 """
 
 import math
@@ -90,21 +89,22 @@ def test_ragged_batch(kernel, H, L, R, dv, g):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("g", [2, 1])
 @pytest.mark.parametrize("workers", [1, 2, 3, 7, 0])
-def test_split_schedule_invariance(kernel, workers):
+def test_split_schedule_invariance(kernel, g, workers):
     """Any number of split-KV workers gives the same result (segments cross workers and sequences)."""
-    d = _case(5, 128, 512, 64, 128, 2, [300, 1, 0, 640, 65], seed=17)
+    d = _case(5, 128, 512, 64, 128, g, [300, 1, 0, 640, 65], seed=17)
     _kernel_or_skip(d, kernel)
     scale = 1 / math.sqrt(192)
     old = tpla.get_option(tpla.OPT_MAX_WORKERS)
     tpla.set_option(tpla.OPT_MAX_WORKERS, workers)
     try:
         got = hx.run_gpu(d, scale, kernel=kernel)
-        got_s = hx.run_gpu(d, scale, mode="shard", shard=1, kernel=kernel)
+        got_s = hx.run_gpu(d, scale, mode="shard", shard=g - 1, kernel=kernel)
     finally:
         tpla.set_option(tpla.OPT_MAX_WORKERS, old)
     hx.assert_close(got, hx.run_oracle(d, scale), "workers=%d" % workers)
-    hx.assert_close(got_s, hx.run_oracle(d, scale, mode="shard", shard=1), "shard workers=%d" % workers)
+    hx.assert_close(got_s, hx.run_oracle(d, scale, mode="shard", shard=g - 1), "shard workers=%d" % workers)
 
 
 # ------------------------------------------------------------------ benchmark configurations, full size
@@ -131,27 +131,35 @@ def test_tpla_g2_dsv3_b1_32k(kernel):
     hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "all shards")
 
 
-def _sampled(d, scale, batch, kernel, modes=("shard", "full")):
+def _every_sequence(d, scale, kernel, modes=("shard", "full"), chunk=4, dev=None):
+    """Every sequence of a full-size case against the oracle (the oracle runs a few sequences at
+    a time so that its float64 copy of the cache stays small)."""
     for mode in modes:
-        got = hx.run_gpu(d, scale, mode=mode, shard=0, kernel=kernel)
-        want = hx.run_oracle(d, scale, mode=mode, shard=0, batch=batch)
-        hx.assert_close(got[batch], want, "%s sampled %s" % (mode, batch))
+        got = hx.run_gpu(d, scale, mode=mode, shard=0, kernel=kernel, dev=dev)
+        for b0 in range(0, d["B"], chunk):
+            batch = list(range(b0, min(d["B"], b0 + chunk)))
+            want = hx.run_oracle(d, scale, mode=mode, shard=0, batch=batch)
+            hx.assert_close(got[batch], want, "%s sequences %d..%d" % (mode, batch[0], batch[-1]))
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
 def test_tpla_g2_dsv3_b16_32k(kernel):
+    """DeepSeek-V3 shape, g = 2, 16 x 32768 tokens; the cache is the oracle's append of seeded raw
+    latents through the Hadamard transform and sliced RMSNorm."""
     spec = gen.WORKLOADS["tpla_g2_dsv3_b16_32k"]
-    d = _case(16, 128, 512, 64, 128, 2, [32768] * 16, 3)
+    d = _case(16, 128, 512, 64, 128, 2, [32768] * 16, 3, transform=ref.TRANSFORM_HADAMARD)
     _kernel_or_skip(d, kernel)
-    _sampled(d, gen.softmax_scale(spec), [0, 9, 15], kernel)
+    _every_sequence(d, gen.softmax_scale(spec), kernel)
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
 def test_tpla_g4_kimi_b8_32k(kernel):
+    """Kimi-K2 shape, g = 4, 8 x 32768 tokens; the cache is the oracle's append through the seeded
+    random orthogonal transform (the PCA stand-in) and sliced RMSNorm."""
     spec = gen.WORKLOADS["tpla_g4_kimi_b8_32k"]
-    d = _case(8, 64, 512, 64, 128, 4, [32768] * 8, 4)
+    d = _case(8, 64, 512, 64, 128, 4, [32768] * 8, 4, transform=ref.TRANSFORM_DENSE)
     _kernel_or_skip(d, kernel)
-    _sampled(d, gen.softmax_scale(spec), [0, 5], kernel)
+    _every_sequence(d, gen.softmax_scale(spec), kernel)
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
@@ -186,22 +194,34 @@ def test_mixed_b64_paged_with_append(kernel):
         g_row = dev["ckv"][page, :, slot].cpu().to(torch.float64).numpy()
         o_row = ckv[page, :, slot]
         assert np.all(np.abs(g_row - o_row) <= np.abs(o_row) * 2.0 ** -7 + 1e-30)
-    # end to end: GPU append + GPU decode against oracle append + oracle decode
-    for mode in ("full", "shard"):
-        got = hx.run_gpu(d_or, scale, mode=mode, shard=0, dev=dev, kernel=kernel)
-        want = hx.run_oracle(d_or, scale, mode=mode, shard=0, batch=batch)
-        hx.assert_close(got[batch], want, "mixed %s" % mode)
+    # end to end: GPU append + GPU decode against oracle append + oracle decode, every sequence
+    _every_sequence(d_or, scale, kernel, modes=("full", "shard"), chunk=8, dev=dev)
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_pv_precision_modes_at_the_length_boundary(kernel):
+@pytest.mark.parametrize("g", [2, 1])
+def test_pv_precision_modes_at_the_length_boundary(kernel, g):
     """Sequences just below 8192 tokens run PV in fp16, from 8192 on in bf16; both meet the tolerance."""
-    d = _case(4, 128, 512, 64, 128, 2, [8191, 8192, 8193, 100], seed=23)
+    d = _case(4, 128, 512, 64, 128, g, [8191, 8192, 8193, 100], seed=23)
     _kernel_or_skip(d, kernel)
     scale = 1 / math.sqrt(192)
     hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "all shards")
-    hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=1, kernel=kernel),
-                    hx.run_oracle(d, scale, mode="shard", shard=1), "shard 1")
+    hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=g - 1, kernel=kernel),
+                    hx.run_oracle(d, scale, mode="shard", shard=g - 1), "shard %d" % (g - 1))
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_mla_g1_dsv3_b8_32k(kernel):
+    """MLA (g = 1) at batch 8 x 32768 tokens, DeepSeek-V3 shape; the cache is the oracle's append
+    through the Hadamard transform and RMSNorm; every sequence against the oracle."""
+    spec = gen.WORKLOADS["mla_g1_dsv3_b8_32k"]
+    d = _case(8, 128, 512, 64, 128, 1, [32768] * 8, 6, transform=ref.TRANSFORM_HADAMARD)
+    _kernel_or_skip(d, kernel)
+    scale = gen.softmax_scale(spec)
+    got = hx.run_gpu(d, scale, mode="mla", kernel=kernel)
+    for b0 in range(0, 8, 4):
+        batch = list(range(b0, b0 + 4))
+        hx.assert_close(got[batch], hx.run_oracle(d, scale, batch=batch), "mla sequences %d.." % b0)
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
@@ -215,3 +235,46 @@ def test_softmax_scale_sign_and_size(kernel, scale):
     hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "scale %g" % scale)
     hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=0, with_wuv=False, kernel=kernel),
                     hx.run_oracle(d, scale, mode="shard", shard=0, with_wuv=False), "scale %g shard latent" % scale)
+
+
+# cache magnitudes at fp16's limits (sequences shorter than 8192 tokens run PV on fp16 tiles, scaled
+# by a power of two where a tile's largest |value| lies outside [2^-10, 65280], and on bf16 tiles
+# where it lies outside [2^-18, 2^23)): name -> (scale of the selected token rows, which rows, scale
+# of the query, rel-RMS bound)
+RANGE_CASES = {
+    "tiny": (2.0 ** -16, "all", 2.0 ** 16, hx.REL_RMS),          # fp16 subnormal range: scaled up by 2^4
+    "huge": (5.0e4, "all", 1.0 / 5.0e4, hx.REL_RMS),              # up to ~2.5e5 > 65504: scaled down by 2^-2
+    "near_max": (1.2e4, "all", 1.0 / 1.2e4, hx.REL_RMS),          # up to ~5.4e4: fits fp16 as it is
+    "mixed_tiny": (2.0 ** -20, "every5", 1.0, hx.REL_RMS),        # a few subnormal rows inside fp16 tiles
+    "mixed_huge": (1.0e5, "every97", 1.0e-5, hx.REL_RMS),         # a few large rows: those tiles scaled down
+    # beyond what a power-of-two shift brings into fp16: bf16 tiles, whose 8-bit P costs about 1e-3
+    # relative error on sequences this short (the documented bound for such caches is 2e-3)
+    "beyond_tiny": (2.0 ** -26, "all", 2.0 ** 26, 2e-3),
+    "beyond_huge": (1.0e9, "all", 1.0e-9, 2e-3),
+}
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("g", [2, 1])
+@pytest.mark.parametrize("case", sorted(RANGE_CASES))
+def test_pv_fp16_range_limits(kernel, g, case):
+    """Latent values whose magnitude fp16 cannot hold (or holds only as subnormals), on sequences
+    short enough for fp16 PV tiles.  Scores are kept ordinary by scaling the query the other way;
+    outputs scale with the cache, so both sides are divided by the row scale before comparing."""
+    row_scale, which, q_scale, rel_bound = RANGE_CASES[case]
+    d = _case(4, 128, 512, 64, 128, g, [300, 1000, 129, 4000], seed=29)
+    _kernel_or_skip(d, kernel)
+    ckv = d["ckv"].to(torch.float32)
+    if which == "all":
+        ckv = ckv * row_scale
+    else:
+        step = int(which[len("every"):])
+        ckv[:, :, ::step, :] *= row_scale                 # every step-th slot of every page
+    d["ckv"] = ckv.to(torch.bfloat16)
+    d["q"] = (d["q"].to(torch.float32) * q_scale).to(torch.bfloat16)
+    scale = 1 / math.sqrt(192)
+    norm = row_scale if which == "all" or row_scale > 1 else 1.0
+    for mode, with_wuv in (("full", True), ("shard", False)):
+        got = hx.run_gpu(d, scale, mode=mode, shard=g - 1, with_wuv=with_wuv, kernel=kernel)
+        want = hx.run_oracle(d, scale, mode=mode, shard=g - 1, with_wuv=with_wuv)
+        hx.assert_close(got / norm, want / norm, "%s %s" % (case, mode), rel_rms=rel_bound)

@@ -18,13 +18,15 @@ from latent_attention_decode_tpla_b200 import tpla
 pytestmark = pytest.mark.gpu
 
 
-def _small():
-    return gen.make_workload(B=3, H=128, L=512, R=64, dv=128, g=2, seq_lens=[100, 64, 300], seed=2, extra_pages=4)
+def _small(g):
+    # g = 2: the 128-token-tile tcgen05 kernel; g = 1 (512 latent columns per shard): the CTA-pair one
+    return gen.make_workload(B=3, H=128, L=512, R=64, dv=128, g=g, seq_lens=[100, 64, 300], seed=2, extra_pages=4)
 
 
+@pytest.mark.parametrize("g", [2, 1])
 @pytest.mark.parametrize("kernel", ["simt", "sm100"])
-def test_bad_page_and_length_are_reported(kernel):
-    d = _small()
+def test_bad_page_and_length_are_reported(kernel, g):
+    d = _small(g)
     if kernel == "sm100" and not hx.sm100_available(d):
         pytest.skip("no tcgen05 variant")
     scale = 1 / math.sqrt(192)
@@ -50,8 +52,9 @@ def test_bad_page_and_length_are_reported(kernel):
         tpla.set_option(tpla.OPT_ATTENTION_KERNEL, old)
 
 
-def test_bounded_wait_times_out_and_context_survives():
-    d = _small()
+@pytest.mark.parametrize("g", [2, 1])
+def test_bounded_wait_times_out_and_context_survives(g):
+    d = _small(g)
     if not hx.sm100_available(d):
         pytest.skip("no tcgen05 variant")
     scale = 1 / math.sqrt(192)

@@ -65,6 +65,41 @@ def test_static_scratch_second_call_with_other_sizes():
             hx.assert_close(o, want, "static scratch after another call")
 
 
+def test_static_scratch_with_fewer_workers_near_its_limit():
+    # 100 sequences x 2 shards: 200 per-sequence partial slots of 128 x 256 fp32 (128 KiB each) plus
+    # the header leave room for only 54 split-KV workers in the 32 MiB array, fewer than the SM
+    # count tpla_decode uses: the result must not change
+    lens = gen.seq_lengths(100, 1, 600, seed=8)
+    d = gen.make_workload(B=100, H=128, L=512, R=64, dv=128, g=2, seq_lens=lens, seed=8, extra_pages=3)
+    want, outs = _decode_both(d, 1 / math.sqrt(192))
+    for o in outs:
+        hx.assert_close(o, want, "static scratch, clamped worker count")
+
+
+def test_static_scratch_kernel_choice_follows_the_options():
+    # the static entry chooses its attention kernel as tpla_decode does: a forced tcgen05 kernel on a
+    # shape without one is rejected, and the kernel that ran is reported
+    d = gen.make_workload(B=2, H=16, L=256, R=32, dv=64, g=2, seq_lens=[100, 7], seed=12)
+    dev = hx.to_device(d)
+    dims = hx.dims_of(d, 0.2)
+    out = torch.zeros(2, 16, 64, dtype=torch.float32, device="cuda")
+    old = tpla.get_option(tpla.OPT_ATTENTION_KERNEL)
+    try:
+        tpla.set_option(tpla.OPT_ATTENTION_KERNEL, 2)
+        with pytest.raises(tpla.TplaError) as e:
+            tpla.decode_static(dims, dev["q"], dev["q_pe"], dev["ckv"], dev["kpe"], dev["block_table"],
+                               dev["seq_lens"], dev["w_uv"], out)
+        assert e.value.status == tpla.TPLA_ERR_UNSUPPORTED
+        tpla.set_option(tpla.OPT_ATTENTION_KERNEL, 1)
+        tpla.decode_static(dims, dev["q"], dev["q_pe"], dev["ckv"], dev["kpe"], dev["block_table"],
+                           dev["seq_lens"], dev["w_uv"], out)
+        torch.cuda.synchronize()
+        assert tpla.get_option(tpla.OPT_LAST_ATTENTION_KERNEL) == 1
+    finally:
+        tpla.set_option(tpla.OPT_ATTENTION_KERNEL, old)
+    assert tpla.check_device_status() == tpla.TPLA_OK
+
+
 def test_static_scratch_rejects_sizes_beyond_its_limit():
     # 1024 sequences x 2 shards of 128 x 256 fp32 partials need 256 MiB > 32 MiB
     d = tpla.make_dims(B=1024, H=128, L=512, R=64, dv=128, g=2, max_pages_per_seq=1, num_pages=1024,
