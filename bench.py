@@ -7,8 +7,10 @@ split-KV attention and the combine (split merge, W_UV, shard sum).  The
 default workload is the DeepSeek-V3 attention shape at TP degree g = 2, one
 rank's share (tpla_decode_shard, shard 0), batch 16, 32768 cached tokens per
 sequence; every input is seeded synthetic data resident in HBM.  The
-per-shard cache (335 MB) is larger than the 126 MB L2, so no L2 flush is
-needed between steps.
+per-shard cache (335 MB) is more than twice the 126 MB L2, so consecutive
+steps read it from HBM; a workload whose cache is smaller keeps several
+replicas of it and each step reads the next one (replicas totalling more than
+twice L2), so that its steps read HBM as well.
 
     python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
 
@@ -35,6 +37,35 @@ if ROOT not in sys.path:
 
 METRIC = "TPLA decode µs/step and latent-cache GB/s (% of B200 HBM peak) at 32K ctx"
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024          # B200 L2
+MIN_TIMED_S = 0.1                     # attention replays are repeated until they span this long
+
+
+def cache_replicas(cache_bytes_per_step):
+    """Cache copies a workload rotates through so that the bytes read between two reads of the same
+    copy exceed twice the L2 (1 when one step already reads that much).  Even, so that the end-to-end
+    leg's double-buffered inputs and the replicas cycle together."""
+    if cache_bytes_per_step > 2 * L2_BYTES:
+        return 1
+    n = 2 * L2_BYTES // max(1, cache_bytes_per_step) + 1
+    return n + (n & 1)
+
+
+def l2_note(replicas, cache_bytes_per_step):
+    if replicas == 1:
+        return "no flush: one step reads %.0f MB of cache, more than twice the 126 MB L2" % (cache_bytes_per_step / 1e6)
+    return "rotated: %d cache replicas, %.0f MB read between two reads of one replica (> 2 x L2)" % (
+        replicas, replicas * cache_bytes_per_step / 1e6)
+
+
+def percentile(xs, q):
+    xs = sorted(xs)
+    if not xs:
+        return float("nan")
+    k = (len(xs) - 1) * q
+    i = int(math.floor(k))
+    j = min(i + 1, len(xs) - 1)
+    return xs[i] + (xs[j] - xs[i]) * (k - i)
 
 
 # ---------------------------------------------------------------- workload description
@@ -59,7 +90,9 @@ def algorithmic_bytes(spec, seq_lens_sum, mode):
 
 # sources that decide what one launch of a kernel does (its code, the shared schedule, the host-side plan)
 KERNEL_SOURCES = {
-    "attn_sm100": ["attn_sm100.cu", "sm100_ptx.cuh", "tpla_internal.cuh", "api.cu"],
+    "attn_sm100": ["attn_sm100.cu", "attn_sm100_common.cuh", "sm100_ptx.cuh", "tpla_internal.cuh", "api.cu"],
+    "attn_sm100_wide": ["attn_sm100_wide.cu", "attn_sm100_common.cuh", "sm100_ptx.cuh", "tpla_internal.cuh",
+                        "api.cu"],
 }
 
 
@@ -206,8 +239,9 @@ def sum_over_ranks(x):
 
 # ---------------------------------------------------------------- GPU arm
 
-def build_device_workload(spec, seed=0):
-    """Seeded synthetic inputs created on the current GPU (bf16 cache N(0,1): unit RMS per shard row)."""
+def build_device_workload(spec, seed=0, replicas=1):
+    """Seeded synthetic inputs created on the current GPU (bf16 cache N(0,1): unit RMS per shard row);
+    ``replicas`` copies of the cache (w["ckvs"], w["kpes"]), the first one also as w["ckv"], w["kpe"]."""
     import torch
     from latent_attention_decode_tpla_b200 import inputs as gen
     from latent_attention_decode_tpla_b200 import tpla
@@ -228,6 +262,10 @@ def build_device_workload(spec, seed=0):
         j = min(num_pages, i + step)
         w["ckv"][i:j] = rn(j - i, g, 64, L // g)
     w["kpe"] = rn(num_pages, 64, R)
+    w["ckvs"], w["kpes"] = [w["ckv"]], [w["kpe"]]
+    for _ in range(1, replicas):
+        w["ckvs"].append(w["ckv"].clone())
+        w["kpes"].append(w["kpe"].clone())
     w["q"] = rn(B, H, L)
     w["q_pe"] = rn(B, H, R)
     w["w_uv"] = rn(H, L, dv, std=1.0 / math.sqrt(L))
@@ -245,29 +283,34 @@ def build_device_workload(spec, seed=0):
     return w
 
 
-def gpu_step(w, spec):
+def gpu_step(w, spec, r=0):
+    """One step on cache replica r: append one token per sequence, attention, combine."""
     from latent_attention_decode_tpla_b200 import tpla
     shard = 0 if spec["mode"] == "shard" else -1
     d = w["dims"]
+    ckv, kpe = w["ckvs"][r], w["kpes"][r]
     tpla.append_kv(d, w["x_new"], w["kpe_new"], spec["transform"], w.get("R_dense"), None, 1e-6,
-                   w["positions"], w["block_table"], w["ckv"], w["kpe"])
-    tpla.attention(d, shard, w["q"], w["q_pe"], w["ckv"], w["kpe"], w["block_table"], w["seq_lens"],
-                   w["workspace"])
+                   w["positions"], w["block_table"], ckv, kpe)
+    tpla.attention(d, shard, w["q"], w["q_pe"], ckv, kpe, w["block_table"], w["seq_lens"], w["workspace"])
     tpla.combine(d, shard, w["seq_lens"], w["w_uv"], w["out"], w["workspace"])
 
 
 def run_gpu_arm(args, spec, rank, world, local):
-    """Times K steps (CUDA events on the launching stream), then K end-to-end steps."""
+    """Times K steps (CUDA events on the launching stream), the attention pass alone over repeated
+    replays (median and p90 per launch), then K end-to-end steps."""
     import torch
     from latent_attention_decode_tpla_b200 import inputs as gen
     from latent_attention_decode_tpla_b200 import tpla
     torch.cuda.set_device(local)
-    w = build_device_workload(spec, seed=0)
+    lens = gen.workload_seq_lens(spec, 0)
+    cache_b, attn_b = algorithmic_bytes(spec, int(lens.sum()), spec["mode"])
+    nrep = cache_replicas(cache_b)
+    w = build_device_workload(spec, seed=0, replicas=nrep)
     if spec["transform"] == 2:
         w["R_dense"] = gen.random_orthogonal(spec["L"], 0).cuda()
     stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        gpu_step(w, spec)
+    for i in range(args.warmup):
+        gpu_step(w, spec, i % nrep)
     torch.cuda.synchronize()
     st = tpla.check_device_status()
     if st != tpla.TPLA_OK:
@@ -275,22 +318,22 @@ def run_gpu_arm(args, spec, rank, world, local):
 
     K = args.steps
     # The timed steps: K steps captured as one CUDA graph and replayed once, so the timed region holds
-    # no host launches.  The attention kernel's own duration comes from a second graph of K
-    # attention launches (the cache is larger than L2, so back-to-back launches read it from HBM).
+    # no host launches; step i reads cache replica i mod nrep.  The attention kernel's own duration
+    # comes from a second graph of K attention launches, replayed several times.
     def capture(fn):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for _ in range(K):
-                fn()
+            for i in range(K):
+                fn(i % nrep)
         g.replay()                                       # untimed: one more warm-up pass
         torch.cuda.synchronize()
         return g
     shard = 0 if spec["mode"] == "shard" else -1
-    g_step = capture(lambda: gpu_step(w, spec))
-    g_attn = capture(lambda: tpla.attention(w["dims"], shard, w["q"], w["q_pe"], w["ckv"], w["kpe"],
-                                            w["block_table"], w["seq_lens"], w["workspace"]))
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g_step = capture(lambda r: gpu_step(w, spec, r))
+    g_attn = capture(lambda r: tpla.attention(w["dims"], shard, w["q"], w["q_pe"], w["ckvs"][r], w["kpes"][r],
+                                              w["block_table"], w["seq_lens"], w["workspace"]))
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    start, end = ev(), ev()
     sampler = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
@@ -299,22 +342,36 @@ def run_gpu_arm(args, spec, rank, world, local):
     g_step.replay()
     end.record(stream)
     torch.cuda.synchronize()
-    clocks = sampler.stop()
     barrier()
-    a0.record(stream)
-    g_attn.replay()
-    a1.record(stream)
-    torch.cuda.synchronize()
+    # attention alone: replays of the K-launch graph, each timed, until they span MIN_TIMED_S (at
+    # least 5), so that the clock sampler sees the load and the spread between replays shows
+    per_launch = []
+    t_total = 0.0
+    while len(per_launch) < 5 or t_total < MIN_TIMED_S * 1e3:
+        a0, a1 = ev(), ev()
+        a0.record(stream)
+        g_attn.replay()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        dt = a0.elapsed_time(a1)
+        t_total += dt
+        per_launch.append(dt / K)
+        if len(per_launch) >= 1000:
+            break
+    clocks = sampler.stop()
     ms = start.elapsed_time(end) / K
-    attn_ms = a0.elapsed_time(a1) / K
+    attn_med = statistics.median(per_launch)
+    attn_p90 = percentile(per_launch, 0.9)
     ms_max = max_over_ranks(ms)
-    attn_ms_max = max_over_ranks(attn_ms)
+    attn_ms_max = max_over_ranks(attn_med)
+    attn_p90_max = max_over_ranks(attn_p90)
 
     # End to end through the public API with host buffers: every step copies its inputs from pinned
     # host memory, runs, and its result is copied back and read on the host.  Consecutive steps are
     # pipelined (inputs and outputs double-buffered on the device, copies on their own streams), so
     # the copies of step i+1's inputs and of step i-1's result overlap step i; each step's kernels
-    # are replayed from a CUDA graph.
+    # are replayed from a CUDA graph (one per cache replica; the replica count is even, so replica
+    # r always uses input buffer r mod 2).
     keys = ("q", "q_pe", "x_new", "kpe_new")
     host = {k: w[k].cpu().pin_memory() for k in keys}
     dev_in = [{k: w[k] for k in keys}, {k: torch.empty_like(w[k]) for k in keys}]
@@ -323,20 +380,19 @@ def run_gpu_arm(args, spec, rank, world, local):
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host[0].numel() * out_host[0].element_size()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
-    # each buffer parity's step (append + attention + combine through the public API) as a CUDA graph,
-    # so that the host issues one replay per step
     graphs = []
-    for sb in range(2):
+    for r in range(max(2, nrep)):
+        sb = r % 2
         wi = dict(w, out=out_dev[sb], **dev_in[sb])
-        gpu_step(wi, spec)                                  # outside capture: one-time setup
+        gpu_step(wi, spec, r % nrep)                        # outside capture: one-time setup
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            gpu_step(wi, spec)
+            gpu_step(wi, spec, r % nrep)
         graphs.append(g)
     torch.cuda.synchronize()
-    ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("in", "done", "out")}
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = {n: [torch.cuda.Event() for _ in range(2)] for n in ("in", "done", "out")}
+    e_start, e_end = ev(), ev()
     torch.cuda.synchronize()
     barrier()
     nsteps = 0 if args.no_e2e else K
@@ -345,25 +401,25 @@ def run_gpu_arm(args, spec, rank, world, local):
         sb = i % 2
         with torch.cuda.stream(up):
             if i >= 2:
-                up.wait_event(ev["done"][sb])           # step i-2 has finished reading these buffers
+                up.wait_event(evs["done"][sb])          # step i-2 has finished reading these buffers
             for k in keys:
                 dev_in[sb][k].copy_(host[k], non_blocking=True)
-            ev["in"][sb].record(up)
-        stream.wait_event(ev["in"][sb])
+            evs["in"][sb].record(up)
+        stream.wait_event(evs["in"][sb])
         if i >= 2:
-            stream.wait_event(ev["out"][sb])            # step i-2's result has left this buffer
+            stream.wait_event(evs["out"][sb])           # step i-2's result has left this buffer
         with torch.cuda.stream(stream):
-            graphs[sb].replay()
-        ev["done"][sb].record(stream)
+            graphs[i % len(graphs)].replay()
+        evs["done"][sb].record(stream)
         with torch.cuda.stream(down):
-            down.wait_event(ev["done"][sb])
+            down.wait_event(evs["done"][sb])
             out_host[sb].copy_(out_dev[sb], non_blocking=True)
-            ev["out"][sb].record(down)
+            evs["out"][sb].record(down)
         if i >= 1:                                      # read step i-1's result on the host
-            ev["out"][(i - 1) % 2].synchronize()
+            evs["out"][(i - 1) % 2].synchronize()
             _ = float(out_host[(i - 1) % 2][0, 0, 0])
     if nsteps:
-        ev["out"][(nsteps - 1) % 2].synchronize()
+        evs["out"][(nsteps - 1) % 2].synchronize()
         _ = float(out_host[(nsteps - 1) % 2][0, 0, 0])
         e_end.record(down)
     else:
@@ -376,11 +432,10 @@ def run_gpu_arm(args, spec, rank, world, local):
         raise RuntimeError("device status after timing: " + tpla.status_string(st))
 
     kernel = tpla.get_option(tpla.OPT_LAST_ATTENTION_KERNEL)
-    cache_b, attn_b = algorithmic_bytes(spec, w["lens_sum"], spec["mode"])
     total_cache = sum_over_ranks(cache_b)
-    return dict(ms=ms_max, attn_ms=attn_ms_max, e2e_ms=e2e_ms, cache_bytes=cache_b, attn_bytes=attn_b,
-                total_cache=total_cache, clocks=clocks, h2d=h2d, d2h=d2h, launches=3 * K, kernel=kernel,
-                lens_sum=w["lens_sum"])
+    return dict(ms=ms_max, attn_ms=attn_ms_max, attn_p90_ms=attn_p90_max, attn_replays=len(per_launch),
+                e2e_ms=e2e_ms, cache_bytes=cache_b, attn_bytes=attn_b, total_cache=total_cache, clocks=clocks,
+                h2d=h2d, d2h=d2h, launches=3 * K, kernel=kernel, lens_sum=w["lens_sum"], replicas=nrep)
 
 
 # ---------------------------------------------------------------- oracle (CPU) arm
@@ -428,10 +483,7 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def cpu_baseline(spec, budget_s=12.0):
-    """Time the oracle on a bounded sample: repeated single-sequence steps until ~budget_s."""
-    s = oracle_sample(spec)
-    cols = (spec["L"] // spec["g"] + spec["R"]) if spec["mode"] == "shard" else (spec["L"] + spec["R"])
+def _time_oracle(spec, s, budget_s):
     t0 = time.perf_counter()
     n = 0
     while True:
@@ -439,11 +491,29 @@ def cpu_baseline(spec, budget_s=12.0):
         n += 1
         if time.perf_counter() - t0 >= budget_s:
             break
-    dt = time.perf_counter() - t0
-    bytes_done = n * s["T"] * cols * 2
-    return {"value": bytes_done / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": "%d oracle step(s) of 1 sequence x %d tokens (%s, all %d heads) in %.1f s; float64 numpy"
-                      % (n, s["T"], "shard 0" if spec["mode"] == "shard" else "all shards", spec["H"], dt)}
+    return n, time.perf_counter() - t0
+
+
+def cpu_baseline(spec, budget_s=12.0, single_core_budget_s=6.0):
+    """Time the oracle on a bounded sample: repeated single-sequence steps until ~budget_s with the
+    BLAS threads of the host, then until ~single_core_budget_s on one thread."""
+    s = oracle_sample(spec)
+    cols = (spec["L"] // spec["g"] + spec["R"]) if spec["mode"] == "shard" else (spec["L"] + spec["R"])
+    n, dt = _time_oracle(spec, s, budget_s)
+    bytes_step = s["T"] * cols * 2
+    out = {"value": n * bytes_step / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": "%d oracle step(s) of 1 sequence x %d tokens (%s, all %d heads) in %.1f s; float64 numpy"
+                     % (n, s["T"], "shard 0" if spec["mode"] == "shard" else "all shards", spec["H"], dt)}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            n1, dt1 = _time_oracle(spec, s, single_core_budget_s)
+        out["single_core"] = {"value": n1 * bytes_step / dt1 / 1e9, "unit": "GB/s", "cores": 1,
+                              "sample": "%d oracle step(s) of the same sequence in %.1f s, BLAS limited to one "
+                                        "thread" % (n1, dt1)}
+    except Exception as e:          # threadpoolctl missing: report why, keep the multi-core figure
+        out["single_core"] = {"unavailable": str(e)}
+    return out
 
 
 def run_reference(args, spec, rank):
@@ -469,7 +539,7 @@ def run_reference(args, spec, rank):
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def config_of(spec):
+def config_of(spec, l2=None):
     T = spec["T"]
     return {"workload": spec["name"], "entry": "tpla_decode_shard(shard 0)" if spec["mode"] == "shard"
             else ("mla_decode" if spec["g"] == 1 else "tpla_decode (all shards, on-chip sum)"),
@@ -478,7 +548,7 @@ def config_of(spec):
             "context": T if not isinstance(T, tuple) else "uniform[%d,%d]" % T,
             "transform": {0: "none", 1: "hadamard", 2: "dense orthogonal (seeded QR)"}[spec["transform"]],
             "page_size": 64, "step": "append 1 token/seq + split-KV attention + combine",
-            "l2": "inputs larger than L2 (no flush)"}
+            "l2": l2 if l2 is not None else "not applicable (oracle on the host)"}
 
 
 # ---------------------------------------------------------------- main
@@ -517,17 +587,19 @@ def main():
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     value = r["total_cache"] / (r["ms"] * 1e-3) / 1e9
     achieved = r["attn_bytes"] / (r["attn_ms"] * 1e-3) / 1e9
-    kernel_name = {1: "attn_simt", 2: "attn_sm100"}.get(r["kernel"], "unknown")
+    kernel_name = {1: "attn_simt", 2: "attn_sm100", 3: "attn_sm100_wide"}.get(r["kernel"], "unknown")
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms"], "us_per_step": r["ms"] * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": config_of(spec),
+        "data": "synthetic", "config": config_of(spec, l2_note(r["replicas"], r["cache_bytes"])),
         "hbm_frac_step": value / world / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(kernel_name, spec["name"]),
                      "kernel": kernel_name + " (tpla_attention)", "peak_kind": peak_kind,
-                     "bytes_per_launch": r["attn_bytes"], "us_per_launch": r["attn_ms"] * 1e3},
+                     "bytes_per_launch": r["attn_bytes"], "us_per_launch": r["attn_ms"] * 1e3,
+                     "us_per_launch_p90": r["attn_p90_ms"] * 1e3, "replays": r["attn_replays"],
+                     "achieved_p90": r["attn_bytes"] / (r["attn_p90_ms"] * 1e-3) / 1e9},
         "e2e": None if args.no_e2e else {
             "value": r["total_cache"] / (r["e2e_ms"] * 1e-3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"]},
