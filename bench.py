@@ -347,7 +347,7 @@ def run_gpu_arm(args, spec, rank, world, local):
     # least 5), so that the clock sampler sees the load and the spread between replays shows
     per_launch = []
     t_total = 0.0
-    while len(per_launch) < 5 or t_total < MIN_TIMED_S * 1e3:
+    while len(per_launch) < 5 or t_total < args.attn_replay_s * 1e3:
         a0, a1 = ev(), ev()
         a0.record(stream)
         g_attn.replay()
@@ -564,6 +564,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
+    ap.add_argument("--tile", type=int, default=0, choices=[0, 64, 128],
+                    help="tokens per tile of the tcgen05 kernel for L/g <= 256 (0: the library default)")
+    ap.add_argument("--attn-replay-s", type=float, default=MIN_TIMED_S,
+                    help="seconds the attention-only replays span at least (5 replays at least)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     spec = workload_spec(args.workload)
@@ -580,6 +584,9 @@ def main():
             print(json.dumps(line), flush=True)
         return
 
+    if args.tile:
+        from latent_attention_decode_tpla_b200 import tpla
+        tpla.set_option(tpla.OPT_TILE_TOKENS, args.tile)
     r = run_gpu_arm(args, spec, rank, world, local)
     if rank != 0:
         return

@@ -272,6 +272,10 @@ int tpla_check_device_status(void* stream);
 #define TPLA_OPT_LAST_ATTENTION_KERNEL 5  /* read-only: kernel of the last attention launch in this
                                              process (0 none yet, 1 CUDA-core, 2 tcgen05 with 128-token
                                              tiles (L/g <= 256), 3 tcgen05 CTA pair (L/g == 512)) */
+#define TPLA_OPT_TILE_TOKENS       6  /* tokens per tile of the tcgen05 kernel for L/g <= 256: 64 (one page per
+                                         tile, more stages in flight) or 128 (two pages, fewer QK^T steps per
+                                         token); 0 = the library's default.  Results are the same up to fp32
+                                         rounding order. */
 int tpla_set_option(int option, int value);
 int tpla_get_option(int option);
 

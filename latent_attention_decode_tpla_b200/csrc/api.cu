@@ -19,15 +19,18 @@ int g_opt_kernel = 0;        // TPLA_OPT_ATTENTION_KERNEL
 int g_opt_max_workers = 0;   // TPLA_OPT_MAX_WORKERS
 int g_opt_wait_limit = 0;    // TPLA_OPT_WAIT_LIMIT
 int g_opt_debug_stall = 0;   // TPLA_OPT_DEBUG_STALL
+int g_opt_tile_tokens = 0;   // TPLA_OPT_TILE_TOKENS
 int g_last_kernel = 0;       // TPLA_OPT_LAST_ATTENTION_KERNEL
 
 // Fewest units a tcgen05 worker gets: keeps the partial traffic small at batch 1.  The CUDA-core
 // kernel is bound by arithmetic, not by that traffic, and spreads the units as widely as it can.
-constexpr int kMinUnitsPerWorker = 6;
+constexpr int kMinUnitsPerWorker = 4;
 // A worker whose range ends one (sequence, shard) and starts the next stops its stream for the
 // first one's epilogue and the second one's query load: measured on B200 at about as long as
 // this many units of streaming.
 constexpr long long kSwitchUnits = 8;
+// Tokens per tile of the tcgen05 kernel for L/g <= 256 (TPLA_OPT_TILE_TOKENS = 0).
+constexpr int kDefaultTileTokens = 128;
 
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mutex;
@@ -127,6 +130,7 @@ int make_plan(const tpla_dims_t* d, int shard, Plan* p) {
     const bool tc = sm100_supports(*p), wide = sm100_wide_supports(*p);
     if (g_opt_kernel == 2 && !tc && !wide) return TPLA_ERR_UNSUPPORTED;
     p->kernel = g_opt_kernel == 1 ? kKernelSimt : (tc ? kKernelSm100 : (wide ? kKernelSm100Wide : kKernelSimt));
+    p->tile_tok = g_opt_tile_tokens ? g_opt_tile_tokens : kDefaultTileTokens;
     // workers: one per SM (a CTA pair per worker for the wide kernel), at most kMaxWorkers
     int cap = p->kernel == kKernelSm100Wide ? sms / 2 : sms;
     cap = cap < kMaxWorkers ? cap : kMaxWorkers;
@@ -348,6 +352,9 @@ int tpla_set_option(int option, int value) {
         case TPLA_OPT_DEBUG_STALL:
             if (value < 0 || value > 1) return TPLA_ERR_INVALID_ARG;
             g_opt_debug_stall = value; return TPLA_OK;
+        case TPLA_OPT_TILE_TOKENS:
+            if (!(value == 0 || value == 64 || value == 128)) return TPLA_ERR_INVALID_ARG;
+            g_opt_tile_tokens = value; return TPLA_OK;
     }
     return TPLA_ERR_INVALID_ARG;
 }
@@ -359,6 +366,7 @@ int tpla_get_option(int option) {
         case TPLA_OPT_WAIT_LIMIT: return g_opt_wait_limit;
         case TPLA_OPT_DEBUG_STALL: return g_opt_debug_stall;
         case TPLA_OPT_LAST_ATTENTION_KERNEL: return g_last_kernel;
+        case TPLA_OPT_TILE_TOKENS: return g_opt_tile_tokens;
     }
     return -1;
 }

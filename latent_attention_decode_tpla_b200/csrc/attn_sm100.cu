@@ -80,34 +80,37 @@ using namespace sm100;
 constexpr int kThreads = 320;
 constexpr int kSoftmaxWarp0 = 2;
 constexpr int kSoftmaxWarps = 8;
-constexpr int kTileTok = 2 * kPage;           // tokens per tile: two pages
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 constexpr int kExactPVBelow = 8192;           // sequences shorter than this run PV in fp16
 constexpr int kPageAhead = 4;                 // page-table entries the producer loads ahead
 
-template <int LS, int RD, int NST>
+template <int LS, int RD, int NST, int TT>
 struct Cfg {
-    static constexpr int kChunk = kTileTok * 128;             // 128 rows x 128 bytes: both pages of a 64-column slice
+    static constexpr int kChunk = TT * 128;                    // TT rows x 128 bytes: a 64-column slice of the tile
     static constexpr int kHalf = kPage * 128;                  // one page's 64 rows of a chunk
     static constexpr int kChunksC = LS / 64;
     static constexpr int kStageBytes = (kChunksC + 1) * kChunk;   // latent chunks + the RoPE chunk
-    static constexpr int kPChunk = 128 * 128;                  // P: 128 rows x 64 tokens x 2 B, two of them
+    static constexpr int kPChunk = 128 * 128;                  // P: 128 rows x 64 tokens x 2 B per chunk
+    static constexpr int kPChunks = TT / 64;
+    static constexpr int kEpiBytes = 32 * 1024 - kPChunks * kPChunk;   // epilogue staging beyond P (8 warps x 4 KB)
+    static constexpr int kCvtShift = TT == 128 ? 10 : 9;       // log2 of the 16-byte pieces of one chunk
     static constexpr int kQpeBytes = 128 * 128;                // RoPE query: 128 rows x 64 x 2 B
     static constexpr int kColO = 0;
     static constexpr int kColS = LS;                           // 128 columns
-    static constexpr int kColQ = LS + kTileTok;                // latent query, LS/2 columns
+    static constexpr int kColQ = LS + TT;                      // latent query, LS/2 columns
     static constexpr int kColsUsed = kColQ + LS / 2;
     static constexpr int kTmemCols = kColsUsed <= 128 ? 128 : (kColsUsed <= 256 ? 256 : 512);
     static constexpr int kStepsC = LS / 16;                    // QK^T steps over the latent
     static constexpr int kStepsR = RD / 16;                    // QK^T steps over the RoPE key
-    static constexpr uint32_t kIdescQK = idesc_f16kind(128, kTileTok, false, true);   // bf16 x bf16
+    static constexpr uint32_t kIdescQK = idesc_f16kind(128, TT, false, true);         // bf16 x bf16
     static constexpr uint32_t kIdescPVf16 = idesc_f16kind(128, LS, true, false);       // fp16 x fp16
     static constexpr uint32_t kIdescPVbf16 = idesc_f16kind(128, LS, true, true);       // bf16 x bf16
-    static constexpr int kCvt = kChunksC * kTileTok * 8 / (kSoftmaxWarps * 32);        // 16-byte pieces per thread
-    static constexpr size_t kSmem = 1024 + (size_t)NST * kStageBytes + 2 * kPChunk + kQpeBytes;
+    static constexpr int kCvt = kChunksC * TT * 8 / (kSoftmaxWarps * 32);              // 16-byte pieces per thread
+    static constexpr size_t kSmem = 1024 + (size_t)NST * kStageBytes + kPChunks * kPChunk + kEpiBytes + kQpeBytes;
     static_assert(kColsUsed <= 512, "tensor memory");
     static_assert(LS % 64 == 0 && RD == 64, "tile shape");
-    static_assert(kCvt >= 1 && kChunksC * kTileTok * 8 % (kSoftmaxWarps * 32) == 0, "conversion split");
+    static_assert(kCvt >= 1 && kChunksC * TT * 8 % (kSoftmaxWarps * 32) == 0, "conversion split");
+    static_assert((TT == 64 || TT == 128) && (1 << kCvtShift) == TT * 8, "tile of one or two pages");
 };
 
 template <int NST>
@@ -124,20 +127,21 @@ struct Bars {
     volatile int abort;
 };
 
-template <int LS, int RD, int NST, bool HALF>
+template <int LS, int RD, int NST, bool HALF, int TT>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_o, Plan p,
                   const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ q_pe,
                   const int32_t* __restrict__ block_table, const int32_t* __restrict__ seq_lens, Workspace ws,
                   uint64_t wait_ns, int debug_stall) {
-    using C = Cfg<LS, RD, NST>;
+    using C = Cfg<LS, RD, NST, TT>;
+    constexpr int kTileTok = TT;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base, by pointer arithmetic on the shared array so that every access
     // derived from it stays a shared-memory access
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    uint8_t* p_smem = smem + NST * C::kStageBytes;          // P: two K chunks of 64 tokens
-    uint8_t* qpe_smem = p_smem + 2 * C::kPChunk;            // RoPE query
+    uint8_t* p_smem = smem + NST * C::kStageBytes;          // P: one K chunk per 64 tokens (+ epilogue staging)
+    uint8_t* qpe_smem = p_smem + C::kPChunks * C::kPChunk + C::kEpiBytes;   // RoPE query
     auto& bars = *reinterpret_cast<Bars<NST>*>(qpe_smem + C::kQpeBytes);
     const uint32_t stage0 = smem_addr(smem);
     const uint32_t p_addr = smem_addr(p_smem);
@@ -235,7 +239,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 }
                 return page;
             };
-            Tile t = make_tile(pos0, lo, lo, hi, 2);
+            Tile t = make_tile(pos0, lo, lo, hi, kTileTok / kPage);
             long long j = 0;
             for (; t.u < hi; ++j) {
                 const int st = (int)(j % NST);
@@ -255,7 +259,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 const uint32_t dst = stage0 + st * C::kStageBytes;
                 mbar_arrive_expect_tx(full, C::kStageBytes);
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
+                for (int k = 0; k < kTileTok / kPage; ++k) {
                     // a missing or invalid page reads rows past the end of the tensor: TMA fills zeros
                     const int page = k == 0 ? page0 : page1;
                     const int yc = page >= 0 ? (page * p.g + shard) * kPage : p.num_pages * p.g * kPage;
@@ -296,7 +300,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             // for the next load.  (Issuing QK^T in several groups, to let a PV that becomes ready
             // meanwhile in sooner, measured much slower on B200: the issue of a group costs far
             // more than its MMAs.)  Each stream has its own tile cursor.
-            Tile tq = make_tile(pos0, lo, lo, hi, 2), tv = tq;
+            Tile tq = make_tile(pos0, lo, lo, hi, kTileTok / kPage), tv = tq;
             long long jq = 0, jv = 0;
             int qseg = -1, vseg = -1;
             bool vbegun = false;
@@ -470,12 +474,14 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             warp_arrive(smem_addr(&bars.q_full));
         };
         if (HALF && upper) {
-            // P rows 64-127 (this warp's lanes, in its warpgroup's K chunk) stay zero
+            // P rows 64-127 (this warp's lanes, in every K chunk) stay zero
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                *reinterpret_cast<uint4*>(p_smem + wg * C::kPChunk + sw128_offset(row, k)) = make_uint4(0, 0, 0, 0);
+            for (int c = 0; c < C::kPChunks; ++c)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<uint4*>(p_smem + c * C::kPChunk + sw128_offset(row, k)) = make_uint4(0, 0, 0, 0);
         }
-        Tile t = make_tile(pos0, lo, lo, hi, 2);
+        Tile t = make_tile(pos0, lo, lo, hi, kTileTok / kPage);
         load_q(pos0);
         long long j = 0;
         for (; t.u < hi; ++j) {
@@ -496,13 +502,21 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             tc_fence_after();
             float s[kCols];
             if (warp_active) {
-#pragma unroll
-                for (int h = 0; h < kCols / 32; ++h) {
-                    uint32_t r[32];
-                    tmem_ld32(lane_base + C::kColS + cbase + 32 * h, r);
+                if constexpr (kCols == 16) {
+                    uint32_t r[16];
+                    tmem_ld16(lane_base + C::kColS + cbase, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) s[32 * h + k] = __uint_as_float(r[k]);
+                    for (int k = 0; k < 16; ++k) s[k] = __uint_as_float(r[k]);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < kCols / 32; ++h) {
+                        uint32_t r[32];
+                        tmem_ld32(lane_base + C::kColS + cbase + 32 * h, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) s[32 * h + k] = __uint_as_float(r[k]);
+                    }
                 }
             } else {
 #pragma unroll
@@ -552,7 +566,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                     const int rr = (i >> 3) & (kTileTok - 1);
                     if (rr < valid) {
                         const uint4 v =
-                            *reinterpret_cast<const uint4*>(sb + (i >> 10) * C::kChunk + rr * 128 + (i & 7) * 16);
+                            *reinterpret_cast<const uint4*>(sb + (i >> C::kCvtShift) * C::kChunk + rr * 128 + (i & 7) * 16);
                         mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
                                                   __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
                     }
@@ -610,7 +624,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 for (int k = 0; k < C::kCvt; ++k) {
                     const int i = tid_sm + k * kSoftmaxWarps * 32;
                     const int rr = (i >> 3) & (kTileTok - 1);
-                    uint4* ptr = reinterpret_cast<uint4*>(sb + (i >> 10) * C::kChunk + rr * 128 + (i & 7) * 16);
+                    uint4* ptr = reinterpret_cast<uint4*>(sb + (i >> C::kCvtShift) * C::kChunk + rr * 128 + (i & 7) * 16);
                     uint4 v = *ptr;
                     if (rr < valid) {
                         v.x = bf16x2_to_f16x2_scaled(v.x, cshift);
@@ -676,10 +690,10 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             // the P buffer is free once PV(j - 1), its last reader, has completed
             if (j >= 1 && !wait_o(j - 1)) break;
             {
-                // this warpgroup's 64 tokens are one K chunk of P; this thread's columns are the
-                // 16-byte pieces from (cbase mod 64) / 8 on, in its head's row
-                uint8_t* pb = p_smem + wg * C::kPChunk;
-                const int k0 = upper ? kCols / 8 : 0;
+                // this thread's columns are the 16-byte pieces from (cbase mod 64) / 8 on, in its
+                // head's row of K chunk cbase / 64 of P (64 tokens per chunk)
+                uint8_t* pb = p_smem + (cbase >> 6) * C::kPChunk;
+                const int k0 = (cbase & 63) >> 3;
 #pragma unroll
                 for (int k = 0; k < kCols / 8; ++k)
                     *reinterpret_cast<uint4*>(pb + sw128_offset(hrow, k0 + k)) =
@@ -710,7 +724,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                     // tensor map and are not written.  Each box waits until the previous store has
                     // read the buffer; the last wait comes before P is written again.
                     const float inv_l = 1.0f / lt;
-                    uint8_t* stile = p_smem + wg * C::kPChunk + quad * 4096;
+                    uint8_t* stile = p_smem + (wg * 4 + quad) * 4096;   // P and the staging beyond it
 #pragma unroll 1
                     for (int c = 0; c < kOHalf / 32; ++c) {
                         uint32_t r[32];
@@ -755,11 +769,11 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
 
 // ------------------------------------------------------------------ host side
 
-template <int LS, int RD, int NST, bool HALF>
+template <int LS, int RD, int NST, bool HALF, int TT>
 cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16* q_pe, const __nv_bfloat16* ckv,
                      const __nv_bfloat16* kpe, const int32_t* bt, const int32_t* seq_lens, Workspace ws,
                      uint64_t wait_ns, int debug_stall, cudaStream_t stream) {
-    using C = Cfg<LS, RD, NST>;
+    using C = Cfg<LS, RD, NST, TT>;
     CUtensorMap tc, tk;
     if (!make_map(&tc, ckv, LS, (uint64_t)p.num_pages * p.g * kPage)) return cudaErrorInvalidValue;
     if (!make_map(&tk, kpe, RD, (uint64_t)p.num_pages * kPage)) return cudaErrorInvalidValue;
@@ -768,7 +782,7 @@ cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16*
     const size_t smem = C::kSmem + sizeof(Bars<NST>);
     static_assert(C::kTmemCols < 512 || C::kSmem > 116 * 1024, "a 512-column TMEM allocation needs one CTA per SM");
     static_assert(C::kSmem + sizeof(Bars<NST>) <= 227 * 1024, "shared memory");
-    auto kern = attn_sm100_kernel<LS, RD, NST, HALF>;
+    auto kern = attn_sm100_kernel<LS, RD, NST, HALF, TT>;
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_once(kern, smem, &attr_done);
     if (e != cudaSuccess) return e;
@@ -788,15 +802,25 @@ cudaError_t launch_attention_sm100(const Plan& p, const __nv_bfloat16* q, const 
                                    int wait_limit_us, int debug_stall, cudaStream_t stream) {
     const uint64_t wait_ns = (wait_limit_us > 0 ? (uint64_t)wait_limit_us : 1000000ull) * 1000ull;
     const bool half = p.H <= 64;
-#define TPLA_LAUNCH(LS, NST)                                                                                       \
-    return half ? launch_t<LS, 64, NST, true>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, \
-                                              stream)                                                              \
-                : launch_t<LS, 64, NST, false>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns, debug_stall, \
-                                               stream)
-    switch (p.Ls) {
-        case 256: TPLA_LAUNCH(256, 2);
-        case 128: TPLA_LAUNCH(128, 3);
-        case 64: TPLA_LAUNCH(64, 5);
+    // stages: as many as fit beside P, the epilogue staging and the RoPE query (two-page tiles: the
+    // 128-token tile of L/g = 256 takes 80 KB; one-page tiles: 40 KB)
+#define TPLA_LAUNCH(LS, NST, TT)                                                                                   \
+    return half ? launch_t<LS, 64, NST, true, TT>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns,         \
+                                                  debug_stall, stream)                                             \
+                : launch_t<LS, 64, NST, false, TT>(p, q, q_pe, ckv, kpe, block_table, seq_lens, ws, wait_ns,        \
+                                                   debug_stall, stream)
+    if (p.tile_tok == 64) {
+        switch (p.Ls) {
+            case 256: TPLA_LAUNCH(256, 4, 64);
+            case 128: TPLA_LAUNCH(128, 7, 64);
+            case 64: TPLA_LAUNCH(64, 10, 64);
+        }
+    } else {
+        switch (p.Ls) {
+            case 256: TPLA_LAUNCH(256, 2, 128);
+            case 128: TPLA_LAUNCH(128, 3, 128);
+            case 64: TPLA_LAUNCH(64, 5, 128);
+        }
     }
 #undef TPLA_LAUNCH
     return cudaErrorNotSupported;

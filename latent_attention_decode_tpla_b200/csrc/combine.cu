@@ -33,11 +33,11 @@ using namespace sm100;
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr size_t kWSmemBudget = 64 * 1024;     // bytes of W_UV staged per CTA
+constexpr size_t kWSmemBudget = 160 * 1024;    // bytes of W_UV staged per CTA (a whole head of 512 x 128 fits)
 constexpr int kMergeTarget = 2048;             // merged floats per CTA the group size aims at
 constexpr int kMaxRows = 8;                    // merged rows projected together, at most
 constexpr int kMaxPairs = 64;                  // (sequence, shard) pairs per CTA
-constexpr int kBatch = 8;                      // segments whose loads a thread issues together
+constexpr int kBatch = 16;                     // segments whose loads a thread issues together
 
 // The schedule's unit boundaries lo(w) = floor(w U / W) and owners, in 32-bit arithmetic when
 // (W + 1) U fits (64-bit integer division is emulated and slow), else in 64 bits.

@@ -42,6 +42,7 @@ struct Plan {
     int max_pages, num_pages;
     int W;             // split-KV workers (a worker of the wide tcgen05 kernel is a CTA pair)
     int kernel;        // attention kernel: kKernelSimt, kKernelSm100 or kKernelSm100Wide
+    int tile_tok;      // tokens per tile of the kKernelSm100 kernel: 64 or 128
     float scale_log2;  // softmax_scale * log2(e)
     unsigned* status;  // device status word (kStatus* bits)
 };

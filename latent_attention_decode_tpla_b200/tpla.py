@@ -33,6 +33,7 @@ OPT_MAX_WORKERS = 2
 OPT_WAIT_LIMIT = 3
 OPT_DEBUG_STALL = 4
 OPT_LAST_ATTENTION_KERNEL = 5
+OPT_TILE_TOKENS = 6
 
 PAGE_SIZE = 64
 

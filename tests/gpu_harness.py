@@ -18,6 +18,22 @@ KERNELS = {"simt": 1, "sm100": 2}
 RAN = {"simt": (1,), "sm100": (2, 3)}
 
 
+class tile_tokens:
+    """Context manager: tokens per tile of the tcgen05 kernel for L/g <= 256 (64, 128; 0 = default)."""
+
+    def __init__(self, tokens):
+        self.tokens = tokens
+
+    def __enter__(self):
+        self.old = tpla.get_option(tpla.OPT_TILE_TOKENS)
+        tpla.set_option(tpla.OPT_TILE_TOKENS, self.tokens)
+        return self
+
+    def __exit__(self, *exc):
+        tpla.set_option(tpla.OPT_TILE_TOKENS, self.old)
+        return False
+
+
 def to64(t):
     return t.detach().to("cpu").to(torch.float64).numpy()
 

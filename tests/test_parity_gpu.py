@@ -22,9 +22,14 @@ pytestmark = pytest.mark.gpu
 KERNELS = ["simt", "sm100"]
 
 
-def _kernel_or_skip(d, kernel):
+def _kernel_or_skip(d, kernel, tile=0):
     if kernel == "sm100" and not hx.sm100_available(d):
         pytest.skip("no tcgen05 variant for this shape")
+    if tile and (kernel != "sm100" or d["L"] // d["g"] > 256):
+        pytest.skip("the tile size is an option of the tcgen05 kernel for L/g <= 256 only")
+
+
+TILES = [0, 64]      # the library default and one-page tiles (two-page tiles when the default is 64)
 
 
 def _case(B, H, L, R, dv, g, lens, seed, transform=None, **kw):
@@ -64,15 +69,21 @@ def test_tiny_g2_hadamard(kernel):
 RAGGED = [0, 1, 63, 64, 65, 200, 7, 129]
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("H,L,R,dv,g", [
     (8, 64, 16, 32, 2), (128, 512, 64, 128, 1), (128, 512, 64, 128, 2), (64, 512, 64, 128, 4),
     (100, 512, 64, 128, 2), (128, 512, 64, 128, 8), (16, 256, 32, 64, 2), (64, 128, 16, 32, 4),
     (32, 512, 64, 128, 2), (64, 512, 64, 128, 8), (48, 512, 64, 128, 2),
 ])
-def test_ragged_batch(kernel, H, L, R, dv, g):
+def test_ragged_batch(kernel, H, L, R, dv, g, tile):
     d = _case(len(RAGGED), H, L, R, dv, g, RAGGED, seed=3 + H + g)
-    _kernel_or_skip(d, kernel)
+    _kernel_or_skip(d, kernel, tile)
+    with hx.tile_tokens(tile):
+        _ragged_batch(d, kernel, H, L, R, dv, g)
+
+
+def _ragged_batch(d, kernel, H, L, R, dv, g):
     scale = 1 / math.sqrt(128 + R)
     want = hx.run_oracle(d, scale)
     hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), want, "out")
@@ -88,21 +99,24 @@ def test_ragged_batch(kernel, H, L, R, dv, g):
                     "identity layout")
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("g", [2, 1])
 @pytest.mark.parametrize("workers", [1, 2, 3, 7, 0])
-def test_split_schedule_invariance(kernel, g, workers):
+def test_split_schedule_invariance(kernel, g, workers, tile):
     """Any number of split-KV workers gives the same result (segments cross workers and sequences)."""
     d = _case(5, 128, 512, 64, 128, g, [300, 1, 0, 640, 65], seed=17)
-    _kernel_or_skip(d, kernel)
+    _kernel_or_skip(d, kernel, tile)
     scale = 1 / math.sqrt(192)
     old = tpla.get_option(tpla.OPT_MAX_WORKERS)
     tpla.set_option(tpla.OPT_MAX_WORKERS, workers)
     try:
+        tpla.set_option(tpla.OPT_TILE_TOKENS, tile)
         got = hx.run_gpu(d, scale, kernel=kernel)
         got_s = hx.run_gpu(d, scale, mode="shard", shard=g - 1, kernel=kernel)
     finally:
         tpla.set_option(tpla.OPT_MAX_WORKERS, old)
+        tpla.set_option(tpla.OPT_TILE_TOKENS, 0)
     hx.assert_close(got, hx.run_oracle(d, scale), "workers=%d" % workers)
     hx.assert_close(got_s, hx.run_oracle(d, scale, mode="shard", shard=g - 1), "shard workers=%d" % workers)
 
@@ -142,33 +156,43 @@ def _every_sequence(d, scale, kernel, modes=("shard", "full"), chunk=4, dev=None
             hx.assert_close(got[batch], want, "%s sequences %d..%d" % (mode, batch[0], batch[-1]))
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_tpla_g2_dsv3_b16_32k(kernel):
+def test_tpla_g2_dsv3_b16_32k(kernel, tile):
     """DeepSeek-V3 shape, g = 2, 16 x 32768 tokens; the cache is the oracle's append of seeded raw
     latents through the Hadamard transform and sliced RMSNorm."""
     spec = gen.WORKLOADS["tpla_g2_dsv3_b16_32k"]
     d = _case(16, 128, 512, 64, 128, 2, [32768] * 16, 3, transform=ref.TRANSFORM_HADAMARD)
-    _kernel_or_skip(d, kernel)
-    _every_sequence(d, gen.softmax_scale(spec), kernel)
+    _kernel_or_skip(d, kernel, tile)
+    with hx.tile_tokens(tile):
+        _every_sequence(d, gen.softmax_scale(spec), kernel)
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_tpla_g4_kimi_b8_32k(kernel):
+def test_tpla_g4_kimi_b8_32k(kernel, tile):
     """Kimi-K2 shape, g = 4, 8 x 32768 tokens; the cache is the oracle's append through the seeded
     random orthogonal transform (the PCA stand-in) and sliced RMSNorm."""
     spec = gen.WORKLOADS["tpla_g4_kimi_b8_32k"]
     d = _case(8, 64, 512, 64, 128, 4, [32768] * 8, 4, transform=ref.TRANSFORM_DENSE)
-    _kernel_or_skip(d, kernel)
-    _every_sequence(d, gen.softmax_scale(spec), kernel)
+    _kernel_or_skip(d, kernel, tile)
+    with hx.tile_tokens(tile):
+        _every_sequence(d, gen.softmax_scale(spec), kernel)
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_mixed_b64_paged_with_append(kernel):
+def test_mixed_b64_paged_with_append(kernel, tile):
     """DeepSeek-V3 shape, g=2: 64 sequences of 1K..64K tokens on a shuffled page table, plus one appended token each."""
     spec = gen.WORKLOADS["tpla_g2_dsv3_b64_mixed"]
     lens = gen.workload_seq_lens(spec, seed=0)
     d = gen.make_workload(B=64, H=128, L=512, R=64, dv=128, g=2, seq_lens=lens, seed=5)
-    _kernel_or_skip(d, kernel)
+    _kernel_or_skip(d, kernel, tile)
+    with hx.tile_tokens(tile):
+        _mixed_b64(d, kernel, spec, lens)
+
+
+def _mixed_b64(d, kernel, spec, lens):
     scale = gen.softmax_scale(spec)
     dev = hx.to_device(d)
     dims = hx.dims_of(d, scale)
@@ -198,16 +222,18 @@ def test_mixed_b64_paged_with_append(kernel):
     _every_sequence(d_or, scale, kernel, modes=("full", "shard"), chunk=8, dev=dev)
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("g", [2, 1])
-def test_pv_precision_modes_at_the_length_boundary(kernel, g):
+def test_pv_precision_modes_at_the_length_boundary(kernel, g, tile):
     """Sequences just below 8192 tokens run PV in fp16, from 8192 on in bf16; both meet the tolerance."""
     d = _case(4, 128, 512, 64, 128, g, [8191, 8192, 8193, 100], seed=23)
-    _kernel_or_skip(d, kernel)
+    _kernel_or_skip(d, kernel, tile)
     scale = 1 / math.sqrt(192)
-    hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "all shards")
-    hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=g - 1, kernel=kernel),
-                    hx.run_oracle(d, scale, mode="shard", shard=g - 1), "shard %d" % (g - 1))
+    with hx.tile_tokens(tile):
+        hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "all shards")
+        hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=g - 1, kernel=kernel),
+                        hx.run_oracle(d, scale, mode="shard", shard=g - 1), "shard %d" % (g - 1))
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
@@ -224,14 +250,21 @@ def test_mla_g1_dsv3_b8_32k(kernel):
         hx.assert_close(got[batch], hx.run_oracle(d, scale, batch=batch), "mla sequences %d.." % b0)
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("g", [2, 1])
 @pytest.mark.parametrize("scale", [-1 / math.sqrt(192), 0.0, 0.5])
-def test_softmax_scale_sign_and_size(kernel, scale):
+def test_softmax_scale_sign_and_size(kernel, scale, g, tile):
     """A negative scale (the kernel folds its sign into the query), a zero scale (uniform
     weights over the valid tokens, ragged tails included) and a large one (the row maximum
     grows by more than the lazy-rescale threshold across tiles)."""
-    d = _case(4, 128, 512, 64, 128, 2, [300, 1, 129, 1000], seed=23)
-    _kernel_or_skip(d, kernel)
+    d = _case(4, 128, 512, 64, 128, g, [300, 1, 129, 1000], seed=23)
+    _kernel_or_skip(d, kernel, tile)
+    with hx.tile_tokens(tile):
+        _scale_case(d, kernel, scale)
+
+
+def _scale_case(d, kernel, scale):
     hx.assert_close(hx.run_gpu(d, scale, kernel=kernel), hx.run_oracle(d, scale), "scale %g" % scale)
     hx.assert_close(hx.run_gpu(d, scale, mode="shard", shard=0, with_wuv=False, kernel=kernel),
                     hx.run_oracle(d, scale, mode="shard", shard=0, with_wuv=False), "scale %g shard latent" % scale)
@@ -254,16 +287,22 @@ RANGE_CASES = {
 }
 
 
+@pytest.mark.parametrize("tile", TILES)
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("g", [2, 1])
 @pytest.mark.parametrize("case", sorted(RANGE_CASES))
-def test_pv_fp16_range_limits(kernel, g, case):
+def test_pv_fp16_range_limits(kernel, g, case, tile):
     """Latent values whose magnitude fp16 cannot hold (or holds only as subnormals), on sequences
     short enough for fp16 PV tiles.  Scores are kept ordinary by scaling the query the other way;
     outputs scale with the cache, so both sides are divided by the row scale before comparing."""
-    row_scale, which, q_scale, rel_bound = RANGE_CASES[case]
     d = _case(4, 128, 512, 64, 128, g, [300, 1000, 129, 4000], seed=29)
-    _kernel_or_skip(d, kernel)
+    _kernel_or_skip(d, kernel, tile)
+    with hx.tile_tokens(tile):
+        _range_case(d, kernel, g, case)
+
+
+def _range_case(d, kernel, g, case):
+    row_scale, which, q_scale, rel_bound = RANGE_CASES[case]
     ckv = d["ckv"].to(torch.float32)
     if which == "all":
         ckv = ckv * row_scale
