@@ -14,8 +14,10 @@ twice L2), so that its steps read HBM as well.
 
     python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
 
-Under torchrun (N > 1) every rank runs an independent replica (the path has
-no exchange step on one node here); the reported time is the max over ranks.
+Under torchrun (N > 1) every rank runs an independent replica by default; the
+reported time is the max over ranks.  With --tp the N ranks are the N shards of
+one tensor-parallel decode (N = the workload's g): each rank appends and decodes
+its shard and the ranks all-reduce their outputs.
 """
 
 import argparse
@@ -204,7 +206,10 @@ def dist_init():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1 and not dist.is_initialized():
         backend = "nccl" if torch.cuda.is_available() else "gloo"
+        backend = os.environ.get("BENCH_DIST_BACKEND", backend)     # gloo: several ranks on one GPU (tests)
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    if torch.cuda.is_available():
+        local = local % torch.cuda.device_count()
     return rank, world, local
 
 
@@ -438,6 +443,98 @@ def run_gpu_arm(args, spec, rank, world, local):
                 h2d=h2d, d2h=d2h, launches=3 * K, kernel=kernel, lens_sum=w["lens_sum"], replicas=nrep)
 
 
+# ---------------------------------------------------------------- tensor-parallel arm
+
+def run_tp_arm(args, spec, rank, world, local):
+    """One TP rank per process (TP degree g = world size, shard = rank): per step, the rank appends its
+    slice of one new token per sequence, decodes its shard and all-reduces the [B, H, dv] output
+    (latent_attention_decode_tpla_b200.tp).  K steps timed between CUDA events on every rank (a CUDA
+    graph when the backend can be captured), the job's time the max over ranks."""
+    import torch
+    import torch.distributed as dist
+    from latent_attention_decode_tpla_b200 import inputs as gen
+    from latent_attention_decode_tpla_b200 import tp, tpla
+    if spec["g"] != world:
+        raise SystemExit("--tp needs the workload's g (%d) processes, got %d" % (spec["g"], world))
+    torch.cuda.set_device(local)
+    B, H, L, R, dv, g = spec["B"], spec["H"], spec["L"], spec["R"], spec["dv"], spec["g"]
+    Ls = L // g
+    lens = gen.workload_seq_lens(spec, 0)
+    maxp = gen.pages_for(int(lens.max()))
+    num_pages = B * maxp
+    gd = torch.Generator(device="cuda")
+    gd.manual_seed(1000 + 77 + rank)
+    rn = lambda *shape, std=1.0: (torch.randn(*shape, generator=gd, device="cuda") * std).to(torch.bfloat16)
+    ckv = torch.empty((num_pages, 64, Ls), dtype=torch.bfloat16, device="cuda")
+    step_rows = max(1, (1 << 27) // (64 * Ls))
+    for i in range(0, num_pages, step_rows):
+        ckv[i:i + step_rows] = rn(min(step_rows, num_pages - i), 64, Ls)
+    kpe = rn(num_pages, 64, R)
+    q_local, q_pe = rn(B, H, Ls), rn(B, H, R)
+    w_local = rn(H, Ls, dv, std=1.0 / math.sqrt(L))
+    x_new, kpe_new = rn(B, L), rn(B, R)
+    bt = gen.block_table(B, maxp, num_pages, 0).cuda()
+    sl = lens.cuda()
+    positions = (lens - 1).clamp(min=0).cuda()
+    dims = tpla.make_dims(B=B, H=H, L=L, R=R, dv=dv, g=g, max_pages_per_seq=maxp, num_pages=num_pages,
+                          softmax_scale=gen.softmax_scale(spec))
+    r = tp.TensorParallelDecode(dims)
+    ws = r.workspace()
+    out = torch.empty((B, H, dv), dtype=torch.float32, device="cuda")
+    R_dense = gen.random_orthogonal(L, 0).cuda() if spec["transform"] == 2 else None
+
+    def step():
+        r.append(x_new, kpe_new, spec["transform"], R_dense, None, 1e-6, positions, bt, ckv, kpe)
+        r.decode(q_local, q_pe, ckv, kpe, bt, sl, w_local, out, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    graph = None
+    if dist.get_backend() == "nccl":
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(K):
+                    step()
+            graph.replay()
+            torch.cuda.synchronize()
+        except Exception:
+            graph = None
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    if graph is not None:
+        graph.replay()
+    else:
+        for _ in range(K):
+            step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / K)
+    st = tpla.check_device_status()
+    if st != tpla.TPLA_OK:
+        raise RuntimeError("device status after timing: " + tpla.status_string(st))
+    timed = "one CUDA graph of K steps" if graph is not None else "K eager steps"
+    del graph                                  # release a graph holding collectives before the group goes
+    cache_rank = int(lens.sum()) * (Ls + R) * 2
+    total = sum_over_ranks(cache_rank)
+    if rank != 0:
+        return None
+    cfg = config_of(spec, "no flush: %.0f MB of cache per rank per step" % (cache_rank / 1e6))
+    cfg.update({"entry": "tensor parallel: per rank tpla_append_kv_shard + tpla_decode (L/g wide) + all_reduce",
+                "parallelism": "tp%d" % world})
+    return {"metric": METRIC, "value": total / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": cfg, "backend": dist.get_backend(),
+            "timed": timed,
+            "gpu_launches": 3 * K}
+
+
 # ---------------------------------------------------------------- oracle (CPU) arm
 
 def oracle_sample(spec, seed=0, T=None):
@@ -564,6 +661,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor parallel across the processes (TP degree = world size = the workload's g)")
     ap.add_argument("--tile", type=int, default=0, choices=[0, 64, 128],
                     help="tokens per tile of the tcgen05 kernel for L/g <= 256 (0: the library default)")
     ap.add_argument("--attn-replay-s", type=float, default=MIN_TIMED_S,
@@ -587,6 +686,11 @@ def main():
     if args.tile:
         from latent_attention_decode_tpla_b200 import tpla
         tpla.set_option(tpla.OPT_TILE_TOKENS, args.tile)
+    if args.tp:
+        line = run_tp_arm(args, spec, rank, world, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     r = run_gpu_arm(args, spec, rank, world, local)
     if rank != 0:
         return

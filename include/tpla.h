@@ -255,6 +255,23 @@ int tpla_append_kv(const tpla_dims_t* dims,
                    tpla_bf16* ckv_cache, tpla_bf16* kpe_cache, void* stream);
 
 /*
+ * tpla_append_kv_shard -- the append of one tensor-parallel rank: the same transform of the whole
+ * new latent x_b and the RMSNorm of shard `shard` (0 <= shard < dims->g) only, written into a cache
+ * that holds that shard alone (TPLA Abstract: each device keeps its slice of the latent):
+ *   ckv_shard_cache [num_pages][64][L/g] bf16: token slot t of page p starts at (p*64 + t) * (L/g)
+ *   kpe_cache       [num_pages][64][R]   bf16 (every rank keeps the whole RoPE key)
+ * Other arguments, results and errors as tpla_append_kv; shard outside [0, g) returns
+ * TPLA_ERR_INVALID_ARG.  A rank then decodes its shard with tpla_decode on dims with L = L/g and
+ * g = 1, its slice q~[:, :, shard*L/g : (shard+1)*L/g] of the absorbed query and its rows of W_UV;
+ * the sum of the ranks' outputs (an all-reduce) is tpla_decode's result on the g-shard cache.
+ */
+int tpla_append_kv_shard(const tpla_dims_t* dims, int shard,
+                         const tpla_bf16* latent_raw, const tpla_bf16* kpe_new,
+                         int transform, const float* R_dense, const float* norm_weight, float eps,
+                         const int32_t* positions, const int32_t* block_table,
+                         tpla_bf16* ckv_shard_cache, tpla_bf16* kpe_cache, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word: TPLA_OK, TPLA_ERR_INDEX or TPLA_ERR_TIMEOUT (or TPLA_ERR_CUDA if the
  * stream reports an error).

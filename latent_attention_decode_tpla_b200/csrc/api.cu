@@ -232,6 +232,34 @@ int run_decode(const tpla_dims_t* d, int shard, const tpla_bf16* q, const tpla_b
     return run_combine(d, shard, seq_lens, w_uv, out, workspace, ws_bytes, stream);
 }
 
+// Cache append of every shard (shard == -1) into the g-shard cache, or of shard `shard` alone into a
+// one-shard cache (one tensor-parallel rank's).
+int run_append(const tpla_dims_t* dims, int shard, const tpla_bf16* latent_raw, const tpla_bf16* kpe_new,
+               int transform, const float* R_dense, const float* norm_weight, float eps, const int32_t* positions,
+               const int32_t* block_table, tpla_bf16* ckv_cache, tpla_bf16* kpe_cache, void* stream) {
+    int st = check_dims(dims);
+    if (st) return st;
+    if (transform < TPLA_TRANSFORM_NONE || transform > TPLA_TRANSFORM_BLOCK_HADAMARD) return TPLA_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return TPLA_ERR_INVALID_ARG;
+    if (dims->B == 0) return TPLA_OK;
+    if (!latent_raw || !kpe_new || !positions || !ckv_cache || !kpe_cache) return TPLA_ERR_INVALID_ARG;
+    if (transform == TPLA_TRANSFORM_DENSE && !R_dense) return TPLA_ERR_INVALID_ARG;
+    if (!aligned16(ckv_cache) || !aligned16(kpe_cache) || !aligned16(latent_raw) || !aligned16(kpe_new))
+        return TPLA_ERR_INVALID_ARG;
+    if (!block_table && (long long)dims->B * dims->max_pages_per_seq > dims->num_pages)
+        return TPLA_ERR_INVALID_ARG;
+    unsigned* status = nullptr;
+    if ((st = device_info(&status, nullptr))) return st;
+    cudaError_t e = launch_append(*dims, shard, reinterpret_cast<const __nv_bfloat16*>(latent_raw),
+                                  reinterpret_cast<const __nv_bfloat16*>(kpe_new), transform, R_dense,
+                                  norm_weight, eps, positions, block_table,
+                                  reinterpret_cast<__nv_bfloat16*>(ckv_cache),
+                                  reinterpret_cast<__nv_bfloat16*>(kpe_cache), status,
+                                  static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return TPLA_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? TPLA_OK : TPLA_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace tpla
 
@@ -300,27 +328,17 @@ int tpla_append_kv(const tpla_dims_t* dims, const tpla_bf16* latent_raw, const t
                    int transform, const float* R_dense, const float* norm_weight, float eps,
                    const int32_t* positions, const int32_t* block_table, tpla_bf16* ckv_cache,
                    tpla_bf16* kpe_cache, void* stream) {
-    int st = check_dims(dims);
-    if (st) return st;
-    if (transform < TPLA_TRANSFORM_NONE || transform > TPLA_TRANSFORM_BLOCK_HADAMARD) return TPLA_ERR_INVALID_ARG;
-    if (!(eps >= 0.f) || !std::isfinite(eps)) return TPLA_ERR_INVALID_ARG;
-    if (dims->B == 0) return TPLA_OK;
-    if (!latent_raw || !kpe_new || !positions || !ckv_cache || !kpe_cache) return TPLA_ERR_INVALID_ARG;
-    if (transform == TPLA_TRANSFORM_DENSE && !R_dense) return TPLA_ERR_INVALID_ARG;
-    if (!aligned16(ckv_cache) || !aligned16(kpe_cache) || !aligned16(latent_raw) || !aligned16(kpe_new))
-        return TPLA_ERR_INVALID_ARG;
-    if (!block_table && (long long)dims->B * dims->max_pages_per_seq > dims->num_pages)
-        return TPLA_ERR_INVALID_ARG;
-    unsigned* status = nullptr;
-    if ((st = device_info(&status, nullptr))) return st;
-    cudaError_t e = launch_append(*dims, reinterpret_cast<const __nv_bfloat16*>(latent_raw),
-                                  reinterpret_cast<const __nv_bfloat16*>(kpe_new), transform, R_dense,
-                                  norm_weight, eps, positions, block_table,
-                                  reinterpret_cast<__nv_bfloat16*>(ckv_cache),
-                                  reinterpret_cast<__nv_bfloat16*>(kpe_cache), status,
-                                  static_cast<cudaStream_t>(stream));
-    if (e == cudaErrorNotSupported) return TPLA_ERR_UNSUPPORTED;
-    return e == cudaSuccess ? TPLA_OK : TPLA_ERR_CUDA;
+    return run_append(dims, -1, latent_raw, kpe_new, transform, R_dense, norm_weight, eps, positions, block_table,
+                      ckv_cache, kpe_cache, stream);
+}
+
+int tpla_append_kv_shard(const tpla_dims_t* dims, int shard, const tpla_bf16* latent_raw,
+                         const tpla_bf16* kpe_new, int transform, const float* R_dense, const float* norm_weight,
+                         float eps, const int32_t* positions, const int32_t* block_table,
+                         tpla_bf16* ckv_shard_cache, tpla_bf16* kpe_cache, void* stream) {
+    if (dims && (shard < 0 || shard >= dims->g)) return TPLA_ERR_INVALID_ARG;
+    return run_append(dims, shard, latent_raw, kpe_new, transform, R_dense, norm_weight, eps, positions, block_table,
+                      ckv_shard_cache, kpe_cache, stream);
 }
 
 int tpla_check_device_status(void* stream) {

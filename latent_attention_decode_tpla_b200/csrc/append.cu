@@ -10,11 +10,12 @@
 //     c_s = y_s / sqrt(mean(y_s^2) + eps)  [* w_s]   for every shard s
 // rounded to bf16 (round to nearest even) and written to
 // ckv[page][s][slot][:], with k_pe copied to kpe[page][slot][:].
-// One CTA per (new token, shard): the Hadamard transform is computed whole in
+// One CTA per (new token, shard of the call): the Hadamard transform is computed whole in
 // every shard's CTA (it mixes all L inputs and costs L log L adds), the dense
 // transform only for the shard's L/g rows, four rows per warp at a time so that
 // many loads of R are in flight.  Each CTA normalises and stores its own
-// slice; the shard-0 CTA also copies k_pe.  Latency-bound: one token per
+// slice; the first CTA of the token also copies k_pe.  A single-shard call (one tensor-parallel
+// rank) computes shard s only and writes it into a cache that holds that shard alone.  Latency-bound: one token per
 // sequence.
 #include "tpla_internal.cuh"
 
@@ -25,7 +26,7 @@ constexpr int kThreads = 512;
 constexpr int kMaxL = 1024;
 
 __global__ void __launch_bounds__(kThreads)
-append_kernel(int L, int R, int g, int max_pages, int num_pages,
+append_kernel(int L, int R, int g, int shard0, int g_out, int max_pages, int num_pages,
               const __nv_bfloat16* __restrict__ latent_raw, const __nv_bfloat16* __restrict__ kpe_new,
               int transform, const float* __restrict__ R_dense, const float* __restrict__ norm_weight,
               float eps, const int32_t* __restrict__ positions, const int32_t* __restrict__ block_table,
@@ -34,7 +35,9 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
     __shared__ float y[kMaxL];
     __shared__ float part[kMaxL / 32];
     __shared__ float inv_rms[8];
-    const int b = blockIdx.x, sh = blockIdx.y, tid = threadIdx.x;
+    // shard sh of the transformed latent goes to shard slot blockIdx.y of a cache laid out with g_out
+    // shards per page (g_out == g: all shards; g_out == 1: one tensor-parallel rank's cache)
+    const int b = blockIdx.x, sh = shard0 + (int)blockIdx.y, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int Ls = L / g;
     // the cache this kernel writes may still be read by the previous kernel (an attention pass)
@@ -43,13 +46,13 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
 
     const int pos = __ldg(positions + b);
     if (pos < 0 || pos >= max_pages * kPage) {
-        if (tid == 0 && sh == 0) atomicOr(status, kStatusIndex);
+        if (tid == 0 && blockIdx.y == 0) atomicOr(status, kStatusIndex);
         return;
     }
     const int lp = pos / kPage;
     const int page = block_table ? __ldg(block_table + (size_t)b * max_pages + lp) : b * max_pages + lp;
-    if (page < 0 || page >= num_pages) {   // recorded once, by the shard-0 CTA
-        if (tid == 0 && sh == 0) atomicOr(status, kStatusIndex);
+    if (page < 0 || page >= num_pages) {   // recorded once, by the first CTA of the token
+        if (tid == 0 && blockIdx.y == 0) atomicOr(status, kStatusIndex);
         return;
     }
     const int slot = pos % kPage;
@@ -161,25 +164,26 @@ append_kernel(int L, int R, int g, int max_pages, int num_pages,
     for (int j = tid; j < Ls; j += kThreads) {
         float v = y[y0 + j] * inv_rms[0];
         if (norm_weight) v *= __ldg(norm_weight + y0 + j);
-        ckv[(((size_t)page * g + sh) * kPage + slot) * Ls + j] = __float2bfloat16_rn(v);
+        ckv[(((size_t)page * g_out + blockIdx.y) * kPage + slot) * Ls + j] = __float2bfloat16_rn(v);
     }
-    if (sh == 0)
+    if (blockIdx.y == 0)
         for (int r = tid; r < R; r += kThreads)
             kpe[((size_t)page * kPage + slot) * R + r] = kpe_new[(size_t)b * R + r];
 }
 
 }  // namespace
 
-cudaError_t launch_append(const tpla_dims_t& d, const __nv_bfloat16* latent_raw,
+cudaError_t launch_append(const tpla_dims_t& d, int shard, const __nv_bfloat16* latent_raw,
                           const __nv_bfloat16* kpe_new, int transform, const float* R_dense,
                           const float* norm_weight, float eps, const int32_t* positions,
                           const int32_t* block_table, __nv_bfloat16* ckv, __nv_bfloat16* kpe,
                           unsigned* status, cudaStream_t stream) {
     if (d.B == 0) return cudaSuccess;
     if (d.L > kMaxL) return cudaErrorNotSupported;
-    return launch_pdl(append_kernel, dim3(d.B, d.g), dim3(kThreads), 0, stream, d.L, d.R, d.g, d.max_pages_per_seq,
-                      d.num_pages, latent_raw, kpe_new, transform, R_dense, norm_weight, eps, positions,
-                      block_table, ckv, kpe, status);
+    const int shard0 = shard < 0 ? 0 : shard, gc = shard < 0 ? d.g : 1;
+    return launch_pdl(append_kernel, dim3(d.B, gc), dim3(kThreads), 0, stream, d.L, d.R, d.g, shard0, gc,
+                      d.max_pages_per_seq, d.num_pages, latent_raw, kpe_new, transform, R_dense, norm_weight, eps,
+                      positions, block_table, ckv, kpe, status);
 }
 
 }  // namespace tpla

@@ -235,7 +235,8 @@ bool sm100_wide_supports(const Plan& p);
 cudaError_t launch_combine(const Plan& p, const int32_t* seq_lens, const __nv_bfloat16* w_uv,
                            float* out, Workspace ws, cudaStream_t stream);
 
-cudaError_t launch_append(const tpla_dims_t& d, const __nv_bfloat16* latent_raw,
+// shard -1: every shard into the g-shard cache; otherwise shard `shard` alone into a one-shard cache
+cudaError_t launch_append(const tpla_dims_t& d, int shard, const __nv_bfloat16* latent_raw,
                           const __nv_bfloat16* kpe_new, int transform, const float* R_dense,
                           const float* norm_weight, float eps, const int32_t* positions,
                           const int32_t* block_table, __nv_bfloat16* ckv, __nv_bfloat16* kpe,

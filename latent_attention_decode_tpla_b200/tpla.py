@@ -40,7 +40,7 @@ PAGE_SIZE = 64
 EXPORTED = ("tpla_status_string", "tpla_decode_workspace_size", "tpla_decode", "tpla_decode_shard",
             "mla_decode", "tpla_attention", "tpla_combine", "tpla_append_kv",
             "tpla_check_device_status", "tpla_set_option", "tpla_get_option", "tpla_version",
-            "tpla_decode_static")
+            "tpla_decode_static", "tpla_append_kv_shard")
 
 
 class Dims(ctypes.Structure):
@@ -86,6 +86,7 @@ def lib():
             "tpla_attention": ([_DIMS, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
             "tpla_combine": ([_DIMS, _I, _P, _P, _P, _P, _SZ, _P], _I),
             "tpla_append_kv": ([_DIMS, _P, _P, _I, _P, _P, _F, _P, _P, _P, _P, _P], _I),
+            "tpla_append_kv_shard": ([_DIMS, _I, _P, _P, _I, _P, _P, _F, _P, _P, _P, _P, _P], _I),
             "tpla_check_device_status": ([_P], _I),
             "tpla_set_option": ([_I, _I], _I),
             "tpla_get_option": ([_I], _I),
@@ -207,6 +208,14 @@ def append_kv(dims, latent_raw, kpe_new, transform, R_dense, norm_weight, eps, p
                                 _f32(R_dense), _f32(norm_weight), float(eps), _i32(positions),
                                 _i32(block_table), _bf16(ckv), _bf16(kpe), _stream(stream)),
            "tpla_append_kv")
+
+
+def append_kv_shard(dims, shard, latent_raw, kpe_new, transform, R_dense, norm_weight, eps, positions,
+                    block_table, ckv_shard, kpe, stream=None):
+    _check(lib().tpla_append_kv_shard(ctypes.byref(dims), int(shard), _bf16(latent_raw), _bf16(kpe_new),
+                                      int(transform), _f32(R_dense), _f32(norm_weight), float(eps),
+                                      _i32(positions), _i32(block_table), _bf16(ckv_shard), _bf16(kpe),
+                                      _stream(stream)), "tpla_append_kv_shard")
 
 
 def check_device_status(stream=None):

@@ -116,6 +116,11 @@ def test_append_validation():
         tpla.TPLA_ERR_INVALID_ARG
     assert L.tpla_append_kv(ctypes.byref(dims(g=3)), *args, 1, None, None, 1e-6, *rest) == \
         tpla.TPLA_ERR_UNSUPPORTED
+    # one tensor-parallel rank's append: the shard must be one of the g shards
+    for shard in (-1, d.g, d.g + 5):
+        assert L.tpla_append_kv_shard(ctypes.byref(d), shard, *args, 1, None, None, 1e-6, *rest) == \
+            tpla.TPLA_ERR_INVALID_ARG
+    assert L.tpla_append_kv_shard(ctypes.byref(d), 0, *args, 7, None, None, 1e-6, *rest) == tpla.TPLA_ERR_INVALID_ARG
 
 
 def test_options_roundtrip():
