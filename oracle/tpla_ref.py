@@ -266,6 +266,34 @@ def decode_shard(q, q_pe, ckv_cache, kpe_cache, block_table, seq_lens, scale, sh
     return project_shards(o, w_uv, [shard])
 
 
+def gla_decode(q, q_pe, ckv_cache, kpe_cache, block_table, seq_lens, scale, *, max_pages_per_seq, w_uv=None):
+    """GLA-style decode, the contrast the edgentiq blog draws in "Introducing TPLA": heads are split
+    into g groups as well as the latent, and head group s (heads s*H/g .. (s+1)*H/g - 1) attends to
+    latent shard s only, with no sum over shards.  Per head h of group s:
+    z_t = scale * (q~_h[s-slice] . c_{t,s} + q_pe_h . k_pe_t), o = softmax(z) C_s, and
+    out_h = W_UV_h[s-rows]^T o (or o itself without w_uv: [B, H, L/g]).  H must be a multiple of g.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    q_pe = np.asarray(q_pe, dtype=np.float64)
+    B, H, L = q.shape
+    g = ckv_cache.shape[1]
+    if H % g:
+        raise ValueError("H must be a multiple of g")
+    Ls, Hg = L // g, H // g
+    w = None if w_uv is None else np.asarray(w_uv, dtype=np.float64)
+    out = np.zeros((B, H, Ls if w is None else w.shape[2]))
+    for b in range(B):
+        T = int(seq_lens[b])
+        if T == 0:
+            continue
+        C, K = gather_sequence(ckv_cache, kpe_cache, block_table, b, T, max_pages_per_seq)
+        for s in range(g):
+            heads = slice(s * Hg, (s + 1) * Hg)
+            _, o = shard_attention(q[b, heads, s * Ls:(s + 1) * Ls], q_pe[b, heads], C[:, s, :], K, scale)
+            out[b, heads] = o if w is None else np.einsum('hl,hld->hd', o, w[heads, s * Ls:(s + 1) * Ls, :])
+    return out
+
+
 def shard_probabilities(q, q_pe, ckv_cache, kpe_cache, block_table, seq_lens, scale, b, s, *,
                         max_pages_per_seq):
     """Softmax weights p [H, T_b] of sequence b on shard s (for invariant checks)."""

@@ -367,6 +367,28 @@ def test_shard_probabilities_match_brute_force():
     assert np.max(np.abs(p0 - p3)) > 1e-3
 
 
+@pytest.mark.parametrize("g", [1, 2, 4])
+def test_gla_decode_matches_brute_force_by_head_group(g):
+    # brute force: each head of group s is the scalar loop of shard s alone (no sum over shards)
+    c = _small_case(B=3, H=4, L=16, R=4, dv=5, g=g, lens=[0, 65, 130], seed=19)
+    scale = 0.33
+    kw = dict(max_pages_per_seq=c["maxp"])
+    got = ref.gla_decode(c["q"], c["q_pe"], c["ckv"], c["kpe"], c["bt"], c["lens"], scale, w_uv=c["w_uv"], **kw)
+    lat = ref.gla_decode(c["q"], c["q_pe"], c["ckv"], c["kpe"], c["bt"], c["lens"], scale, **kw)
+    Hg = 4 // g
+    for s in range(g):
+        heads = slice(s * Hg, (s + 1) * Hg)
+        np.testing.assert_allclose(got[:, heads], _brute_force(c, scale, shard_only=s)[:, heads], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lat[:, heads], _brute_force(c, scale, shard_only=s, latent=True)[:, heads],
+                                   rtol=0, atol=1e-12)
+    if g == 1:   # one group: MLA
+        np.testing.assert_allclose(got, ref.decode(c["q"], c["q_pe"], c["ckv"], c["kpe"], c["bt"], c["lens"], scale,
+                                                   w_uv=c["w_uv"], **kw), rtol=0, atol=1e-13)
+    if g > 1:   # heads must split evenly into the groups
+        with pytest.raises(ValueError):
+            ref.gla_decode(c["q"][:, :3], c["q_pe"][:, :3], c["ckv"], c["kpe"], c["bt"], c["lens"], scale, **kw)
+
+
 def _to_g1(ckv):
     n, g, _, Ls = ckv.shape
     return ckv.transpose(0, 2, 1, 3).reshape(n, P, g * Ls)[:, None]

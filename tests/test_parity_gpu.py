@@ -317,3 +317,29 @@ def _range_case(d, kernel, g, case):
         got = hx.run_gpu(d, scale, mode=mode, shard=g - 1, with_wuv=with_wuv, kernel=kernel)
         want = hx.run_oracle(d, scale, mode=mode, shard=g - 1, with_wuv=with_wuv)
         hx.assert_close(got / norm, want / norm, "%s %s" % (case, mode), rel_rms=rel_bound)
+
+
+# ------------------------------------------------------------------ GLA-style decode (heads split with the latent)
+
+@pytest.mark.parametrize("H,g", [(128, 2), (64, 4), (128, 1)])
+def test_gla_style_decode(H, g):
+    """Head group s attends to latent shard s only (the contrast on the TPLA pages): the library's
+    kernels per group against the oracle's GLA-style decode, with and without W_UV."""
+    from latent_attention_decode_tpla_b200 import gla
+    d = _case(len(RAGGED), H, 512, 64, 128, g, RAGGED, seed=61 + g)
+    scale = 1 / math.sqrt(192)
+    dev = hx.to_device(d)
+    dims = hx.dims_of(d, scale)
+    bt = d["block_table"].numpy()
+    kw = dict(max_pages_per_seq=d["max_pages_per_seq"])
+    f = lambda t: hx.to64(t)
+    for with_wuv in (True, False):
+        cols = 128 if with_wuv else 512 // g
+        out = torch.full((len(RAGGED), H, cols), float("nan"), dtype=torch.float32, device="cuda")
+        gla.gla_decode(dims, dev["q"], dev["q_pe"], dev["ckv"], dev["kpe"], dev["block_table"], dev["seq_lens"],
+                       dev["w_uv"] if with_wuv else None, out)
+        torch.cuda.synchronize()
+        assert tpla.check_device_status() == tpla.TPLA_OK
+        want = ref.gla_decode(f(d["q"]), f(d["q_pe"]), f(d["ckv"]), f(d["kpe"]), bt, d["seq_lens"].numpy(), scale,
+                              w_uv=f(d["w_uv"]) if with_wuv else None, **kw)
+        hx.assert_close(hx.to64(out), want, "gla H=%d g=%d w_uv=%s" % (H, g, with_wuv))
