@@ -52,11 +52,12 @@
 // to a polynomial on the FMA pipe measured slower here, since the softmax is
 // bound by its latency chain, not by that unit's throughput.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads into a ring of NST
+// Warp roles (384 threads): warp 0 issues TMA loads into a ring of NST
 // stages (page-table entries fetched a few pages ahead); warp 1 allocates
 // tensor memory and issues the MMAs from one thread, polling for whichever
-// of QK^T(next tile) and PV(oldest tile) is ready; warps 2-9 are two softmax
-// warpgroups.  Both own all 128 TMEM lanes (one head row per thread);
+// of QK^T(next tile) and PV(oldest tile) is ready; warps 2-3 only complete
+// the control warpgroup, whose registers go to the softmax; warps 4-11 are
+// two softmax warpgroups.  Both own all 128 TMEM lanes (one head row per thread);
 // warpgroup 0 takes score columns 0-63 of every tile, warpgroup 1 columns
 // 64-127, and they agree on each row's running maximum through a per-tile
 // exchange.  Each warpgroup rescales, and finally writes, its half of the O
@@ -77,8 +78,17 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
-constexpr int kSoftmaxWarp0 = 2;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxWarp0 = 4;                // warps 4-11: two whole hardware warpgroups
+// Register split.  Ten or twelve warps on four sub-partitions put three warps on some of them, which
+// caps a thread at 168 registers, and the softmax path spills at that cap.  The control warpgroup
+// (warps 0-3; the MMA issue code needs about 120) gives the rest of its share to the softmax
+// warpgroups: launched at 168 per thread (64,512 registers), 4 warps x 120 + 8 warps x 192 per lane
+// adds up to that total exactly, and neither side spills.
+constexpr int kLaunchRegs = 168;
+constexpr int kCtrlRegs = 120;
+constexpr int kSoftmaxRegs = 192;
+static_assert(32 * (4 * kCtrlRegs + 8 * kSoftmaxRegs) <= kLaunchRegs * kThreads, "register split");
 constexpr int kSoftmaxWarps = 8;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 constexpr int kExactPVBelow = 8192;           // sequences shorter than this run PV in fp16
@@ -198,193 +208,201 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     const uint32_t tmem = bars.tmem_base;
     // 2 cycles per nanosecond bounds the clock from above (B200 runs at most 1.965 GHz)
     const Waiter wt{&bars.abort, p.status, wait_ns * 2};
-
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            // Page-table entries are loaded kPageAhead units ahead of their TMA issue, as plain
-            // loads that can all be in flight at once; an entry is checked when it is used.
-            // (Prefetching the units a stage ring ahead into L2 measured slower on B200.)
-            UnitPos ahead = pos0;
-            long long ua = lo;
-            auto raw_page = [&](const UnitPos& u) -> int {
-                return block_table ? __ldg(block_table + (size_t)u.b * p.max_pages + u.tile)
-                                   : u.b * p.max_pages + u.tile;
-            };
-            int pg[kPageAhead];
-#pragma unroll
-            for (int k = 0; k < kPageAhead; ++k) {
-                pg[k] = -1;
-                if (ua < hi) {
-                    pg[k] = raw_page(ahead);
-                    advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
-                    ++ua;
+    // Each role's code sits inside the branch that set its register budget, so that the compiler
+    // allocates it within that budget.
+    if (warp < kSoftmaxWarp0) {
+        reg_dealloc<kCtrlRegs>();
+        if (warp == 0) {
+            // ------------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                // Page-table entries are loaded kPageAhead units ahead of their TMA issue, as plain
+                // loads that can all be in flight at once; an entry is checked when it is used.
+                // (Prefetching the units a stage ring ahead into L2 measured slower on B200.)
+                UnitPos ahead = pos0;
+                long long ua = lo;
+                auto raw_page = [&](const UnitPos& u) -> int {
+                    return block_table ? __ldg(block_table + (size_t)u.b * p.max_pages + u.tile)
+                                       : u.b * p.max_pages + u.tile;
+                };
+                int pg[kPageAhead];
+    #pragma unroll
+                for (int k = 0; k < kPageAhead; ++k) {
+                    pg[k] = -1;
+                    if (ua < hi) {
+                        pg[k] = raw_page(ahead);
+                        advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
+                        ++ua;
+                    }
+                }
+                // every popped entry belongs to a unit of the range: an entry outside [0, num_pages)
+                // is a caller error, recorded, and the page reads as zeros
+                auto pop_page = [&]() -> int {
+                    int page = pg[0];
+                    if (page < 0 || page >= p.num_pages) {
+                        atomicOr(p.status, kStatusIndex);
+                        page = -1;
+                    }
+    #pragma unroll
+                    for (int k = 0; k + 1 < kPageAhead; ++k) pg[k] = pg[k + 1];
+                    pg[kPageAhead - 1] = -1;
+                    if (ua < hi) {
+                        pg[kPageAhead - 1] = raw_page(ahead);
+                        advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
+                        ++ua;
+                    }
+                    return page;
+                };
+                Tile t = make_tile(pos0, lo, lo, hi, kTileTok / kPage);
+                long long j = 0;
+                for (; t.u < hi; ++j) {
+                    const int st = (int)(j % NST);
+                    const uint32_t use = (uint32_t)(j / NST);
+                    const int page0 = pop_page();
+                    const int page1 = t.npages == 2 ? pop_page() : -1;
+                    if (use > 0 && !wt.wait(smem_addr(&bars.empty[st]), (use - 1) & 1)) break;
+                    const int shard = p.shard0 + t.pos.s;
+                    if (t.begin && j > 0) {
+                        // the softmax warps load this segment's query when the previous segment's last
+                        // tile is done, a few tiles from now: have it in L2 by then
+                        const __nv_bfloat16* qrow = q + (size_t)t.pos.b * p.H * p.L + (size_t)shard * LS;
+                        for (int h = 0; h < p.H; ++h) prefetch_l2(qrow + (size_t)h * p.L, LS * 2);
+                        prefetch_l2(q_pe + (size_t)t.pos.b * p.H * RD, (uint32_t)(p.H * RD * 2));
+                    }
+                    const uint32_t full = smem_addr(&bars.full[st]);
+                    const uint32_t dst = stage0 + st * C::kStageBytes;
+                    mbar_arrive_expect_tx(full, C::kStageBytes);
+    #pragma unroll
+                    for (int k = 0; k < kTileTok / kPage; ++k) {
+                        // a missing or invalid page reads rows past the end of the tensor: TMA fills zeros
+                        const int page = k == 0 ? page0 : page1;
+                        const int yc = page >= 0 ? (page * p.g + shard) * kPage : p.num_pages * p.g * kPage;
+                        const int yk = page >= 0 ? page * kPage : p.num_pages * kPage;
+    #pragma unroll
+                        for (int c = 0; c < C::kChunksC; ++c)
+                            tma_load_2d(dst + c * C::kChunk + k * C::kHalf, &tm_c, full, c * 64, yc);
+                        tma_load_2d(dst + C::kChunksC * C::kChunk + k * C::kHalf, &tm_k, full, 0, yk);
+                    }
+                    t = next_tile(t, seq_lens, p, lo, hi);
+                }
+                // All loads are issued: the next kernel (the combine) may launch once every CTA is
+                // here.  Triggering at the start instead lets its CTAs pile onto the SMs whose workers
+                // finish first, which unbalances the combine.
+                pdl_trigger();
+                // drain: the last use of every stage must have landed before the CTA exits
+                for (long long x = j - NST < 0 ? 0 : j - NST; x < j; ++x) {
+                    const int st = (int)(x % NST);
+                    // bounded wait that ignores the abort flag (the copy is in flight either way)
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(smem_addr(&bars.full[st]), (uint32_t)(x / NST) & 1)) {
+                        if (globaltimer_ns() - t0 > wait_ns) {
+                            atomicOr(p.status, kStatusTimeout);
+                            break;
+                        }
+                    }
                 }
             }
-            // every popped entry belongs to a unit of the range: an entry outside [0, num_pages)
-            // is a caller error, recorded, and the page reads as zeros
-            auto pop_page = [&]() -> int {
-                int page = pg[0];
-                if (page < 0 || page >= p.num_pages) {
-                    atomicOr(p.status, kStatusIndex);
-                    page = -1;
+            __syncwarp();
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                bool ok = true;
+                if (debug_stall) ok = wt.wait(smem_addr(&bars.never), 0);   // nothing arrives: exercises the time-out
+                // Issue whichever MMA is ready, polling without blocking: PV of the oldest tile as soon
+                // as its P is in shared memory, QK^T of the next tile as soon as its stage has landed
+                // and S has been read.  PV goes first when both are ready, since it releases a stage
+                // for the next load.  (Issuing QK^T in several groups, to let a PV that becomes ready
+                // meanwhile in sooner, measured much slower on B200: the issue of a group costs far
+                // more than its MMAs.)  Each stream has its own tile cursor.
+                Tile tq = make_tile(pos0, lo, lo, hi, kTileTok / kPage), tv = tq;
+                long long jq = 0, jv = 0;
+                int qseg = -1, vseg = -1;
+                bool vbegun = false, vexact = false;
+                long long idle_since = clock64();
+                while (ok && tv.u < hi) {
+                    bool did = false;
+                    if (jv < jq) {
+                        if (tv.begin && !vbegun) {
+                            ++vseg;
+                            vexact = tv.pos.T < kExactPVBelow;
+                            vbegun = true;
+                        }
+                        if (mbar_test_wait(smem_addr(&bars.p_full), (uint32_t)(jv & 1)) &&
+                            (!tv.begin || vseg == 0 ||
+                             mbar_test_wait(smem_addr(&bars.o_free), (uint32_t)((vseg - 1) & 1)))) {
+                            tc_fence_after();
+                            const int st = (int)(jv % NST);
+                            const uint32_t sb = stage0 + st * C::kStageBytes;
+                            // a short segment's softmax warps chose this tile's PV type before they
+                            // signalled P; a long segment's tiles are bf16
+                            const uint32_t idesc_pv =
+                                vexact && bars.pv_f16[jv & 1] ? C::kIdescPVf16 : C::kIdescPVbf16;
+    #pragma unroll
+                            for (int kk = 0; kk < kTileTok / 16; ++kk) {
+                                // A: 16 tokens of P (K-major); B: the same 16 token rows of every latent chunk (MN-major)
+                                const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * C::kPChunk + (kk & 3) * 32, 16, 1024);
+                                const uint64_t bd = smem_desc_sw128(sb + kk * 2048, C::kChunk, 1024);
+                                mma_ss(tmem + C::kColO, ad, bd, idesc_pv, (tv.begin && kk == 0) ? 0u : 1u);
+                            }
+                            mma_commit(smem_addr(&bars.empty[st]));
+                            mma_commit(smem_addr(&bars.o_done));
+                            tv = next_tile(tv, seq_lens, p, lo, hi);
+                            ++jv;
+                            vbegun = false;
+                            did = true;
+                        }
+                    }
+                    if (tq.u < hi) {
+                        const int st = (int)(jq % NST);
+                        if ((!tq.begin || mbar_test_wait(smem_addr(&bars.q_full), (uint32_t)((qseg + 1) & 1))) &&
+                            mbar_test_wait(smem_addr(&bars.full[st]), (uint32_t)((jq / NST) & 1)) &&
+                            (jq == 0 || mbar_test_wait(smem_addr(&bars.s_free), (uint32_t)((jq - 1) & 1)))) {
+                            if (tq.begin) ++qseg;
+                            tc_fence_after();
+                            const uint32_t sb = stage0 + st * C::kStageBytes;
+                            const uint32_t d = tmem + C::kColS;
+    #pragma unroll
+                            for (int kk = 0; kk < C::kStepsC; ++kk) {
+                                const uint64_t bd = smem_desc_sw128(sb + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024);
+                                mma_ts(d, tmem + C::kColQ + kk * 8, bd, C::kIdescQK, kk > 0 ? 1u : 0u);
+                            }
+    #pragma unroll
+                            for (int kk = 0; kk < C::kStepsR; ++kk) {
+                                const uint64_t ad = smem_desc_sw128(qpe_addr + kk * 32, 16, 1024);
+                                const uint64_t bd = smem_desc_sw128(sb + C::kChunksC * C::kChunk + kk * 32, 16, 1024);
+                                mma_ss(d, ad, bd, C::kIdescQK, 1u);
+                            }
+                            mma_commit(smem_addr(&bars.s_full));
+                            tq = next_tile(tq, seq_lens, p, lo, hi);
+                            ++jq;
+                            did = true;
+                        }
+                    }
+                    if (did) {
+                        idle_since = clock64();
+                    } else {
+                        if (bars.abort) break;
+                        if ((uint64_t)(clock64() - idle_since) > wt.limit_cycles) {
+                            atomicOr(p.status, kStatusTimeout);
+                            bars.abort = 1;
+                            break;
+                        }
+                    }
                 }
-#pragma unroll
-                for (int k = 0; k + 1 < kPageAhead; ++k) pg[k] = pg[k + 1];
-                pg[kPageAhead - 1] = -1;
-                if (ua < hi) {
-                    pg[kPageAhead - 1] = raw_page(ahead);
-                    advance_unit(ahead, seq_lens, p.B, p.max_pages, p.gc);
-                    ++ua;
-                }
-                return page;
-            };
-            Tile t = make_tile(pos0, lo, lo, hi, kTileTok / kPage);
-            long long j = 0;
-            for (; t.u < hi; ++j) {
-                const int st = (int)(j % NST);
-                const uint32_t use = (uint32_t)(j / NST);
-                const int page0 = pop_page();
-                const int page1 = t.npages == 2 ? pop_page() : -1;
-                if (use > 0 && !wt.wait(smem_addr(&bars.empty[st]), (use - 1) & 1)) break;
-                const int shard = p.shard0 + t.pos.s;
-                if (t.begin && j > 0) {
-                    // the softmax warps load this segment's query when the previous segment's last
-                    // tile is done, a few tiles from now: have it in L2 by then
-                    const __nv_bfloat16* qrow = q + (size_t)t.pos.b * p.H * p.L + (size_t)shard * LS;
-                    for (int h = 0; h < p.H; ++h) prefetch_l2(qrow + (size_t)h * p.L, LS * 2);
-                    prefetch_l2(q_pe + (size_t)t.pos.b * p.H * RD, (uint32_t)(p.H * RD * 2));
-                }
-                const uint32_t full = smem_addr(&bars.full[st]);
-                const uint32_t dst = stage0 + st * C::kStageBytes;
-                mbar_arrive_expect_tx(full, C::kStageBytes);
-#pragma unroll
-                for (int k = 0; k < kTileTok / kPage; ++k) {
-                    // a missing or invalid page reads rows past the end of the tensor: TMA fills zeros
-                    const int page = k == 0 ? page0 : page1;
-                    const int yc = page >= 0 ? (page * p.g + shard) * kPage : p.num_pages * p.g * kPage;
-                    const int yk = page >= 0 ? page * kPage : p.num_pages * kPage;
-#pragma unroll
-                    for (int c = 0; c < C::kChunksC; ++c)
-                        tma_load_2d(dst + c * C::kChunk + k * C::kHalf, &tm_c, full, c * 64, yc);
-                    tma_load_2d(dst + C::kChunksC * C::kChunk + k * C::kHalf, &tm_k, full, 0, yk);
-                }
-                t = next_tile(t, seq_lens, p, lo, hi);
-            }
-            // All loads are issued: the next kernel (the combine) may launch once every CTA is
-            // here.  Triggering at the start instead lets its CTAs pile onto the SMs whose workers
-            // finish first, which unbalances the combine.
-            pdl_trigger();
-            // drain: the last use of every stage must have landed before the CTA exits
-            for (long long x = j - NST < 0 ? 0 : j - NST; x < j; ++x) {
-                const int st = (int)(x % NST);
-                // bounded wait that ignores the abort flag (the copy is in flight either way)
+                // drain every MMA this thread issued before tensor memory is freed
+                mma_commit(smem_addr(&bars.drain));
                 const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(smem_addr(&bars.full[st]), (uint32_t)(x / NST) & 1)) {
+                while (!mbar_try_wait(smem_addr(&bars.drain), 0)) {
                     if (globaltimer_ns() - t0 > wait_ns) {
                         atomicOr(p.status, kStatusTimeout);
                         break;
                     }
                 }
             }
+            __syncwarp();
         }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            bool ok = true;
-            if (debug_stall) ok = wt.wait(smem_addr(&bars.never), 0);   // nothing arrives: exercises the time-out
-            // Issue whichever MMA is ready, polling without blocking: PV of the oldest tile as soon
-            // as its P is in shared memory, QK^T of the next tile as soon as its stage has landed
-            // and S has been read.  PV goes first when both are ready, since it releases a stage
-            // for the next load.  (Issuing QK^T in several groups, to let a PV that becomes ready
-            // meanwhile in sooner, measured much slower on B200: the issue of a group costs far
-            // more than its MMAs.)  Each stream has its own tile cursor.
-            Tile tq = make_tile(pos0, lo, lo, hi, kTileTok / kPage), tv = tq;
-            long long jq = 0, jv = 0;
-            int qseg = -1, vseg = -1;
-            bool vbegun = false;
-            long long idle_since = clock64();
-            while (ok && tv.u < hi) {
-                bool did = false;
-                if (jv < jq) {
-                    if (tv.begin && !vbegun) {
-                        ++vseg;
-                        vbegun = true;
-                    }
-                    if (mbar_test_wait(smem_addr(&bars.p_full), (uint32_t)(jv & 1)) &&
-                        (!tv.begin || vseg == 0 ||
-                         mbar_test_wait(smem_addr(&bars.o_free), (uint32_t)((vseg - 1) & 1)))) {
-                        tc_fence_after();
-                        const int st = (int)(jv % NST);
-                        const uint32_t sb = stage0 + st * C::kStageBytes;
-                        // the softmax warps chose this tile's PV type before they signalled P
-                        const uint32_t idesc_pv = bars.pv_f16[jv & 1] ? C::kIdescPVf16 : C::kIdescPVbf16;
-#pragma unroll
-                        for (int kk = 0; kk < kTileTok / 16; ++kk) {
-                            // A: 16 tokens of P (K-major); B: the same 16 token rows of every latent chunk (MN-major)
-                            const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * C::kPChunk + (kk & 3) * 32, 16, 1024);
-                            const uint64_t bd = smem_desc_sw128(sb + kk * 2048, C::kChunk, 1024);
-                            mma_ss(tmem + C::kColO, ad, bd, idesc_pv, (tv.begin && kk == 0) ? 0u : 1u);
-                        }
-                        mma_commit(smem_addr(&bars.empty[st]));
-                        mma_commit(smem_addr(&bars.o_done));
-                        tv = next_tile(tv, seq_lens, p, lo, hi);
-                        ++jv;
-                        vbegun = false;
-                        did = true;
-                    }
-                }
-                if (tq.u < hi) {
-                    const int st = (int)(jq % NST);
-                    if ((!tq.begin || mbar_test_wait(smem_addr(&bars.q_full), (uint32_t)((qseg + 1) & 1))) &&
-                        mbar_test_wait(smem_addr(&bars.full[st]), (uint32_t)((jq / NST) & 1)) &&
-                        (jq == 0 || mbar_test_wait(smem_addr(&bars.s_free), (uint32_t)((jq - 1) & 1)))) {
-                        if (tq.begin) ++qseg;
-                        tc_fence_after();
-                        const uint32_t sb = stage0 + st * C::kStageBytes;
-                        const uint32_t d = tmem + C::kColS;
-#pragma unroll
-                        for (int kk = 0; kk < C::kStepsC; ++kk) {
-                            const uint64_t bd = smem_desc_sw128(sb + (kk >> 2) * C::kChunk + (kk & 3) * 32, 16, 1024);
-                            mma_ts(d, tmem + C::kColQ + kk * 8, bd, C::kIdescQK, kk > 0 ? 1u : 0u);
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < C::kStepsR; ++kk) {
-                            const uint64_t ad = smem_desc_sw128(qpe_addr + kk * 32, 16, 1024);
-                            const uint64_t bd = smem_desc_sw128(sb + C::kChunksC * C::kChunk + kk * 32, 16, 1024);
-                            mma_ss(d, ad, bd, C::kIdescQK, 1u);
-                        }
-                        mma_commit(smem_addr(&bars.s_full));
-                        tq = next_tile(tq, seq_lens, p, lo, hi);
-                        ++jq;
-                        did = true;
-                    }
-                }
-                if (did) {
-                    idle_since = clock64();
-                } else {
-                    if (bars.abort) break;
-                    if ((uint64_t)(clock64() - idle_since) > wt.limit_cycles) {
-                        atomicOr(p.status, kStatusTimeout);
-                        bars.abort = 1;
-                        break;
-                    }
-                }
-            }
-            // drain every MMA this thread issued before tensor memory is freed
-            mma_commit(smem_addr(&bars.drain));
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(smem_addr(&bars.drain), 0)) {
-                if (globaltimer_ns() - t0 > wait_ns) {
-                    atomicOr(p.status, kStatusTimeout);
-                    break;
-                }
-            }
-        }
-        __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax / epilogue (warps 2..9)
+        reg_alloc<kSoftmaxRegs>();
+        // ------------------------------------------------------------ softmax / epilogue (warps 4..11)
         const int sw = warp - kSoftmaxWarp0;              // 0..7
         const int wg = sw >> 2;                           // which half of the tile columns and of O
         const int quad = warp & 3;
@@ -598,6 +616,11 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
 #pragma unroll
                 for (int k = 0; k < kCols; ++k) l4[k & 3] += s[k];
                 lt = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                // a long segment's tiles are bf16 without a vote: pack here, beside the exponentials
+                if (!exact) pack();
+            } else {
+#pragma unroll
+                for (int k = 0; k < kCols / 2; ++k) pk[k] = 0u;
             }
             if (exact) {
                 if (!wt.wait(smem_addr(&bars.vote), (uint32_t)(nvote & 1))) break;
@@ -609,12 +632,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 f16 = pv_fp16_shift(tmax, e);
                 cshift = __int_as_float((127 + e) << 23);
                 pshift = __int_as_float((127 - e) << 23);
-            }
-            if (warp_active) {
-                pack();
-            } else {
-#pragma unroll
-                for (int k = 0; k < kCols / 2; ++k) pk[k] = 0u;
+                if (warp_active) pack();
             }
             if (f16) {
                 // this tile's latent rows -> fp16 (rows past the sequence end -> 0) for PV;
@@ -699,7 +717,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                     *reinterpret_cast<uint4*>(pb + sw128_offset(hrow, k0 + k)) =
                         make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
             }
-            if (tid_sm == 0) bars.pv_f16[j & 1] = f16 ? 1 : 0;   // read by the issuer after p_full
+            if (exact && tid_sm == 0) bars.pv_f16[j & 1] = f16 ? 1 : 0;   // read by the issuer after p_full
             fence_proxy_async_smem();
             warp_arrive(smem_addr(&bars.p_full));
             first_tile = false;
@@ -786,6 +804,17 @@ cudaError_t launch_t(const Plan& p, const __nv_bfloat16* q, const __nv_bfloat16*
     static unsigned long long attr_done = 0;
     cudaError_t e = set_smem_once(kern, smem, &attr_done);
     if (e != cudaSuccess) return e;
+    // The register split draws on the registers the CTA is launched with: a build that gives the
+    // kernel fewer than kLaunchRegs per thread would leave the softmax warps waiting for registers
+    // that never come, so it is refused here.
+    static int regs_ok = -1;
+    if (regs_ok < 0) {
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        regs_ok = fa.numRegs >= kLaunchRegs ? 1 : 0;
+    }
+    if (!regs_ok) return cudaErrorNotSupported;
     return launch_pdl(kern, dim3(p.W), dim3(kThreads), smem, stream, tc, tk, to, p, q, q_pe, bt, seq_lens, ws,
                       wait_ns, debug_stall);
 }
