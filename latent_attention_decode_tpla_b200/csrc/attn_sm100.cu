@@ -577,17 +577,22 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
             bool f16 = false;
             float cshift = 1.f, pshift = 1.f;             // 2^e for the latent tile, 2^-e for P
             if (exact) {
+                // all of this thread's loads in flight at once; rows past the sequence end are
+                // loaded (they lie inside the stage) but not counted
                 uint32_t mx = 0;
-#pragma unroll 4
+                uint4 vt[C::kCvt];
+#pragma unroll
                 for (int k = 0; k < C::kCvt; ++k) {
                     const int i = tid_sm + k * kSoftmaxWarps * 32;
                     const int rr = (i >> 3) & (kTileTok - 1);
-                    if (rr < valid) {
-                        const uint4 v =
-                            *reinterpret_cast<const uint4*>(sb + (i >> C::kCvtShift) * C::kChunk + rr * 128 + (i & 7) * 16);
-                        mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                                                  __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
-                    }
+                    vt[k] = *reinterpret_cast<const uint4*>(sb + (i >> C::kCvtShift) * C::kChunk + rr * 128 + (i & 7) * 16);
+                }
+#pragma unroll
+                for (int k = 0; k < C::kCvt; ++k) {
+                    const int rr = ((tid_sm + k * kSoftmaxWarps * 32) >> 3) & (kTileTok - 1);
+                    if (rr < valid)
+                        mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(vt[k].x & 0x7FFF7FFFu, vt[k].y & 0x7FFF7FFFu),
+                                                  __vmaxu2(vt[k].z & 0x7FFF7FFFu, vt[k].w & 0x7FFF7FFFu)));
                 }
                 mx = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
                 if (lane == 0) bars.vote_max[nvote & 1][sw] = mx;
