@@ -131,6 +131,13 @@ int make_plan(const tpla_dims_t* d, int shard, Plan* p) {
     if (g_opt_kernel == 2 && !tc && !wide) return TPLA_ERR_UNSUPPORTED;
     p->kernel = g_opt_kernel == 1 ? kKernelSimt : (tc ? kKernelSm100 : (wide ? kKernelSm100Wide : kKernelSimt));
     p->tile_tok = g_opt_tile_tokens ? g_opt_tile_tokens : kDefaultTileTokens;
+    // split-KV cost weights: a tile of a sequence shorter than 8192 tokens takes the tcgen05
+    // kernels' fp16 PV path (a range vote and an in-place conversion of the tile), measured at
+    // about 1.3x the cost of a long sequence's tile; the CUDA-core kernel has one cost
+    const bool tc_kernel = p->kernel == kKernelSm100 || p->kernel == kKernelSm100Wide;
+    p->w_long = tc_kernel ? 3 : 1;
+    p->w_short = tc_kernel ? 4 : 1;
+    p->short_below = tc_kernel ? 8192 : 0;
     // workers: one per SM (a CTA pair per worker for the wide kernel), at most kMaxWorkers
     int cap = p->kernel == kKernelSm100Wide ? sms / 2 : sms;
     cap = cap < kMaxWorkers ? cap : kMaxWorkers;

@@ -93,9 +93,10 @@ attn_simt_kernel(Plan p, const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     // CTAs of this one have exited (no early trigger)
     pdl_wait();
 
-    const long long U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
-    if (U == 0) return;
-    const long long lo = unit_lo(w, U, p.W), hi = unit_lo(w + 1, U, p.W);
+    const long long V = warp_total_weight(seq_lens, p);
+    if (V == 0) return;
+    const long long lo = warp_unit_at_weight(seq_lens, p, unit_lo(w, V, p.W));
+    const long long hi = warp_unit_at_weight(seq_lens, p, unit_lo(w + 1, V, p.W));
     if (lo >= hi) {
         // a worker with no units leaves a zero-weight partial in its slot: the merge may count it
         // as a segment of the pair it falls inside
@@ -225,8 +226,7 @@ attn_simt_kernel(Plan p, const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
         }
         if (seg_end) {
             // the segment started at max(lo, unit of tile 0 of this (b, s))
-            const long long seg_first = u - pos.tile < lo ? lo : u - pos.tile;
-            const int sl = (seg_first == lo) ? w : p.W + pos.b * p.gc + pos.s;
+            const int sl = u - pos.tile >= lo ? p.W + pos.b * p.gc + pos.s : w;
             __syncthreads();
 #pragma unroll
             for (int a = 0; a < C::kHpt; ++a) {

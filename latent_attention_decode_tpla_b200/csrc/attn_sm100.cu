@@ -187,9 +187,10 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
     pdl_wait();
 
     // every warp derives the same unit range from seq_lens
-    const long long U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
-    if (U == 0) return;
-    const long long lo = unit_lo(w, U, p.W), hi = unit_lo(w + 1, U, p.W);
+    const long long V = warp_total_weight(seq_lens, p);
+    if (V == 0) return;
+    const long long lo = warp_unit_at_weight(seq_lens, p, unit_lo(w, V, p.W));
+    const long long hi = warp_unit_at_weight(seq_lens, p, unit_lo(w + 1, V, p.W));
     if (lo >= hi) {
         // a worker with no units leaves a zero-weight partial in its slot: the merge may count it
         // as a segment of the pair it falls inside
@@ -738,8 +739,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constan
                 float lt = l + bars.xsum_buf[seg & 1][wg ^ 1][row];
                 if (HALF) lt += bars.xsum_buf[seg & 1][wg][row ^ 64] + bars.xsum_buf[seg & 1][wg ^ 1][row ^ 64];
                 const long long u_first = t.u - pos.tile;       // unit of page 0 of this (b, s)
-                const long long seg_first = u_first < lo ? lo : u_first;
-                const int slot = seg_first == lo ? w : p.W + pos.b * p.gc + pos.s;
+                const int slot = u_first >= lo ? p.W + pos.b * p.gc + pos.s : w;
                 if (o_warp) {
                     // The normalised rows go out 32 columns at a time: staged in this warp's own
                     // rows of the P buffer (free: the segment's last PV has completed), 128B-swizzled,

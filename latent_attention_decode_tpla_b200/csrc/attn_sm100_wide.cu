@@ -141,9 +141,10 @@ attn_wide_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
     // every input may have been written by the previous kernel on the stream: wait for it
     pdl_wait();
 
-    const long long U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
-    if (U == 0) return;
-    const long long lo = unit_lo(w, U, p.W), hi = unit_lo(w + 1, U, p.W);
+    const long long V = warp_total_weight(seq_lens, p);
+    if (V == 0) return;
+    const long long lo = warp_unit_at_weight(seq_lens, p, unit_lo(w, V, p.W));
+    const long long hi = warp_unit_at_weight(seq_lens, p, unit_lo(w + 1, V, p.W));
     if (lo >= hi) {
         // a worker with no units leaves a zero-weight partial in its slot (see attn_sm100.cu)
         if (half == 0)
@@ -607,8 +608,7 @@ attn_wide_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
                 if (!wt.wait(smem_addr(&bars.xsum), (uint32_t)(seg & 1))) break;
                 const float lsum = l + bars.xsum_buf[seg & 1][wg ^ 1][row];
                 const long long u_first = t.u - pos.tile;
-                const long long seg_first = u_first < lo ? lo : u_first;
-                const int slot = seg_first == lo ? w : p.W + pos.b * p.gc + pos.s;
+                const int slot = u_first >= lo ? p.W + pos.b * p.gc + pos.s : w;
                 if (warp_active) {
                     // normalised rows out 32 columns at a time, staged (128B-swizzled) in this warp's
                     // 4 KB of the query region -- free: the segment's last QK^T has completed -- and

@@ -39,23 +39,21 @@ constexpr int kMaxRows = 8;                    // merged rows projected together
 constexpr int kMaxPairs = 64;                  // (sequence, shard) pairs per CTA
 constexpr int kBatch = 16;                     // segments whose loads a thread issues together
 
-// The schedule's unit boundaries lo(w) = floor(w U / W) and owners, in 32-bit arithmetic when
-// (W + 1) U fits (64-bit integer division is emulated and slow), else in 64 bits.
+// The owner of the unit whose weighted start is v (the largest w with floor(w V / W) <= v), in
+// 32-bit arithmetic when (W + 1) V fits (64-bit integer division is emulated and slow), else in 64
+// bits.
 struct UnitMath {
-    long long U;
+    long long V;
     int W;
     bool small;
-    __device__ long long lo(long long w) const {
-        return small ? (long long)(((unsigned)w * (unsigned)U) / (unsigned)W) : unit_lo(w, U, W);
-    }
-    __device__ int worker(long long u) const {
-        return small ? (int)(((unsigned)(u + 1) * (unsigned)W - 1u) / (unsigned)U) : unit_worker(u, U, W);
+    __device__ int worker(long long v) const {
+        return small ? (int)(((unsigned)(v + 1) * (unsigned)W - 1u) / (unsigned)V) : unit_worker(v, V, W);
     }
 };
 
 struct PairInfo {
     int wf, wl;        // workers holding the pair's first and last tile (wl < wf: empty sequence)
-    int first_slot;    // slot of the first segment
+    int first_slot;    // slot of the first segment (the one that starts at tile 0)
 };
 
 template <int kRows>
@@ -95,37 +93,39 @@ combine_kernel(Plan p, int Bc, int dsub, const int32_t* __restrict__ seq_lens, W
                           smem_addr(&wbar));
         }
     }
-    // 2. first and last worker of each pair: prefix sum of tiles over the sequences before b
+    // 2. first and last worker of each pair: prefix sum of the unit weights over the sequences
+    // before b (the schedule in tpla_internal.cuh)
     if (warp == (project ? 1 : 0)) {
         UnitMath um;
-        um.U = warp_total_units(seq_lens, p.B, p.max_pages, p.gc);
+        um.V = warp_total_weight(seq_lens, p);
         um.W = p.W;
-        um.small = um.U < (1ll << 32) / (p.W + 1);
-        long long before = 0;                         // units of sequences < base
+        um.small = um.V < (1ll << 32) / (p.W + 1);
+        long long before = 0;                         // weight of sequences < base
         for (int base = 0; base < b0 + nb; base += 32) {
             const int b = base + lane;
-            int nt = 0;
+            int nt = 0, c = 1;
             if (b < b0 + nb) {
                 int T = __ldg(seq_lens + b);
                 T = T < 0 ? 0 : (T > p.max_pages * kPage ? p.max_pages * kPage : T);
                 nt = tiles_of_len(T);
+                c = unit_weight(p, T);
             }
-            long long incl = (long long)nt * p.gc;   // inclusive scan over the lanes
+            long long incl = (long long)nt * p.gc * c;   // inclusive scan over the lanes
             for (int o = 1; o < 32; o <<= 1) {
                 const long long v = __shfl_up_sync(0xffffffffu, incl, o);
                 if (lane >= o) incl += v;
             }
             if (b >= b0 && b < b0 + nb) {
-                const long long ub = before + incl - (long long)nt * p.gc;   // first unit of sequence b
+                const long long vb = before + incl - (long long)nt * p.gc * c;   // weighted start of b
                 for (int s = 0; s < p.gc; ++s) {
                     PairInfo pi;
                     if (nt == 0) {
                         pi.wf = 0; pi.wl = -1; pi.first_slot = 0;
                     } else {
-                        const long long u0 = ub + (long long)s * nt;
-                        pi.wf = um.worker(u0);
-                        pi.wl = um.worker(u0 + nt - 1);
-                        pi.first_slot = um.lo(pi.wf) == u0 ? pi.wf : p.W + b * p.gc + s;
+                        const long long v0 = vb + (long long)s * nt * c;
+                        pi.wf = um.worker(v0);
+                        pi.wl = um.worker(v0 + (long long)(nt - 1) * c);
+                        pi.first_slot = p.W + b * p.gc + s;
                     }
                     pinfo[(b - b0) * p.gc + s] = pi;
                 }

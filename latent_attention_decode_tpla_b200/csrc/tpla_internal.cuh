@@ -3,12 +3,16 @@
 // Split-KV schedule (not on the TPLA pages; it is how one GPU keeps all SMs
 // busy at small batch): the work of a call is a list of "units", one per
 // (sequence b, shard s of the call, 64-token tile), ordered b-major, then
-// shard, then tile.  Worker w (a CTA, or a CTA pair) takes the contiguous
-// unit range [lo(w), lo(w+1)) with lo(w) = floor(w * U / W).  Inside that
-// range each run of one (b, s) is a "segment"; it leaves one partial result
-// (normalised output rows + log2-sum-exp per head) in slot
-//     w                      if the segment starts the worker's range,
-//     W + b * gc + s         otherwise (the segment then starts at tile 0).
+// shard, then tile.  Each unit has a cost weight, the same for all units of
+// one sequence: the tcgen05 kernels spend more per tile on a sequence short
+// enough for fp16 PV tiles (Plan::w_short against Plan::w_long).  With V the
+// total weight and Vpos(u) the weight of the units before u, worker w (a CTA,
+// or a CTA pair) takes the units whose Vpos lies in [v(w), v(w+1)),
+// v(w) = floor(w * V / W): a contiguous unit range [lo(w), lo(w+1)).  Inside
+// that range each run of one (b, s) is a "segment"; it leaves one partial
+// result (normalised output rows + log2-sum-exp per head) in slot
+//     W + b * gc + s         if the segment starts at tile 0 of (b, s),
+//     w                      otherwise (it then starts the worker's range).
 // The combine kernel rebuilds the same lists from seq_lens alone, so the host
 // never needs the lengths and no kernel waits on another CTA.
 #pragma once
@@ -43,6 +47,8 @@ struct Plan {
     int W;             // split-KV workers (a worker of the wide tcgen05 kernel is a CTA pair)
     int kernel;        // attention kernel: kKernelSimt, kKernelSm100 or kKernelSm100Wide
     int tile_tok;      // tokens per tile of the kKernelSm100 kernel: 64 or 128
+    int w_long, w_short;   // split-KV cost weight of a unit of a sequence of >= / < short_below tokens
+    int short_below;
     float scale_log2;  // softmax_scale * log2(e)
     unsigned* status;  // device status word (kStatus* bits)
 };
@@ -104,6 +110,62 @@ __device__ inline long long warp_total_units(const int32_t* seq_lens, int B, int
     }
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     return acc * gc;
+}
+
+// Cost weight of each unit of a sequence of T tokens (the split-KV schedule above).
+__host__ __device__ inline int unit_weight(const Plan& p, int T) { return T < p.short_below ? p.w_short : p.w_long; }
+
+// Sum over b of gc * tiles(b) * weight(b), by one full warp (all 32 lanes call it).
+__device__ inline long long warp_total_weight(const int32_t* seq_lens, const Plan& p) {
+    const int lane = threadIdx.x & 31;
+    long long acc = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        if (b < p.B) {
+            int T = __ldg(seq_lens + b);
+            T = T < 0 ? 0 : (T > p.max_pages * kPage ? p.max_pages * kPage : T);
+            acc += (long long)tiles_of_len(T) * unit_weight(p, T);
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    return acc * p.gc;
+}
+
+// The first unit (plain index) whose weighted start Vpos(u) is >= v, by one full warp; the total
+// unit count when there is none.
+__device__ inline long long warp_unit_at_weight(const int32_t* seq_lens, const Plan& p, long long v) {
+    const int lane = threadIdx.x & 31;
+    long long ubefore = 0, vbefore = 0;         // units and weight of sequences < base
+    for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        long long n = 0;
+        int c = 1;
+        if (b < p.B) {
+            int T = __ldg(seq_lens + b);
+            T = T < 0 ? 0 : (T > p.max_pages * kPage ? p.max_pages * kPage : T);
+            n = (long long)tiles_of_len(T) * p.gc;
+            c = unit_weight(p, T);
+        }
+        long long un = n, vn = n * c;           // inclusive scans over the 32 lanes
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long a = __shfl_up_sync(0xffffffffu, un, o), bb = __shfl_up_sync(0xffffffffu, vn, o);
+            if (lane >= o) { un += a; vn += bb; }
+        }
+        const long long vchunk = __shfl_sync(0xffffffffu, vn, 31);
+        if (v < vbefore + vchunk) {
+            // the first sequence whose weighted range ends past v holds the answer (or the next)
+            const unsigned hit = __ballot_sync(0xffffffffu, b < p.B && v < vbefore + vn);
+            const int src = __ffs(hit) - 1;
+            const long long vs = vbefore + __shfl_sync(0xffffffffu, vn - n * c, src);   // its weighted start
+            const long long us = ubefore + __shfl_sync(0xffffffffu, un - n, src);       // its first unit
+            const int cs = __shfl_sync(0xffffffffu, c, src);
+            const long long k = v <= vs ? 0 : (v - vs + cs - 1) / cs;                   // units before v's unit
+            return us + k;
+        }
+        ubefore += __shfl_sync(0xffffffffu, un, 31);
+        vbefore += vchunk;
+    }
+    return ubefore;
 }
 
 // Position of unit u in (b, s, tile) coordinates, found by one full warp.
