@@ -294,6 +294,30 @@ def gla_decode(q, q_pe, ckv_cache, kpe_cache, block_table, seq_lens, scale, *, m
     return out
 
 
+def mla_prefill(latent_raw, kpe_new, q, q_pe, scale, *, transform=TRANSFORM_HADAMARD, R_dense=None,
+                norm_weight=None, eps=1e-6, w_uv=None):
+    """Prefill of one prompt in MLA form ([BLOG] "Prefill-Decode Separation": prefill keeps MLA, decode uses
+    TPLA): every head attends over the whole latent, normalised by one RMSNorm over all L columns.
+
+    latent_raw [T, L] pre-norm latents and kpe_new [T, R] RoPE keys of the prompt's tokens; q [T, H, L]
+    absorbed queries and q_pe [T, H, R], all in the transformed basis.  The latent rows are the g = 1
+    append rounded like the cache, c_i = bf16(R x_i / sqrt(mean((R x_i)^2) + eps)); token t attends
+    causally: z_i = scale * (q~_t . c_i + q_pe_t . k_pe_i) for i <= t, o_t = softmax(z) C, and
+    out_t = W_UV^T o_t (o_t itself without w_uv).  Returns [T, H, dv] or [T, H, L].
+    """
+    c = bf16_round(append_values(latent_raw, 1, transform, R_dense, norm_weight, eps))[:, 0, :]   # [T, L]
+    K = np.asarray(kpe_new, dtype=np.float64)
+    q = np.asarray(q, dtype=np.float64)
+    q_pe = np.asarray(q_pe, dtype=np.float64)
+    T, H, L = q.shape
+    w = None if w_uv is None else np.asarray(w_uv, dtype=np.float64)
+    out = np.zeros((T, H, L if w is None else w.shape[2]))
+    for t in range(T):
+        _, o = shard_attention(q[t], q_pe[t], c[:t + 1], K[:t + 1], scale)
+        out[t] = o if w is None else np.einsum('hl,hld->hd', o, w)
+    return out
+
+
 def shard_probabilities(q, q_pe, ckv_cache, kpe_cache, block_table, seq_lens, scale, b, s, *,
                         max_pages_per_seq):
     """Softmax weights p [H, T_b] of sequence b on shard s (for invariant checks)."""

@@ -440,3 +440,65 @@ def test_tokens_past_seq_len_are_ignored():
     ckv[page, :, 6:, :] = 1e6      # slots 70.. of the tail page
     b = ref.decode(c["q"], c["q_pe"], ckv, c["kpe"], c["bt"], c["lens"], 0.7, w_uv=c["w_uv"], **kw)
     np.testing.assert_array_equal(a, b)
+
+
+# ---------------------------------------------------------------- MLA-form prefill
+
+def test_mla_prefill_matches_brute_force():
+    # independent statement: Sylvester H_8 from scipy, one RMSNorm over the whole row, bf16 by torch's
+    # cast, then scalar loops for the causal softmax and the W_UV projection
+    rng = np.random.default_rng(17)
+    T, H, L, R, dv = 5, 2, 8, 4, 3
+    x = rng.standard_normal((T, L))
+    kpe = np.asarray(torch.from_numpy(rng.standard_normal((T, R))).to(torch.bfloat16).to(torch.float64))
+    q = rng.standard_normal((T, H, L))
+    q_pe = rng.standard_normal((T, H, R))
+    w = rng.standard_normal((H, L, dv))
+    scale, eps = 0.37, 1e-6
+    Hm = scipy.linalg.hadamard(L) / math.sqrt(L)
+    c = []
+    for t in range(T):
+        y = Hm @ x[t]
+        y = y / math.sqrt(sum(v * v for v in y) / L + eps)
+        c.append(torch.tensor(y).to(torch.bfloat16).to(torch.float64).numpy())
+    want = np.zeros((T, H, dv))
+    for t in range(T):
+        for h in range(H):
+            zs = [scale * (sum(q[t, h, j] * c[i][j] for j in range(L)) + sum(q_pe[t, h, r] * kpe[i, r] for r in range(R)))
+                  for i in range(t + 1)]
+            m = max(zs)
+            es = [math.exp(z - m) for z in zs]
+            den = sum(es)
+            for d in range(dv):
+                want[t, h, d] = sum(es[i] / den * sum(c[i][j] * w[h, j, d] for j in range(L)) for i in range(t + 1))
+    got = ref.mla_prefill(x, kpe, q, q_pe, scale, transform=ref.TRANSFORM_HADAMARD, eps=eps, w_uv=w)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    # the first token sees only itself: out_0 = W_UV^T c_0 for every head
+    np.testing.assert_allclose(got[0], np.einsum('l,hld->hd', c[0], w), rtol=1e-12, atol=1e-12)
+    # without W_UV the rows are convex combinations of the latent rows seen so far
+    lat = ref.mla_prefill(x, kpe, q, q_pe, scale, transform=ref.TRANSFORM_HADAMARD, eps=eps)
+    np.testing.assert_allclose(lat[0], np.broadcast_to(c[0], (H, L)), rtol=1e-12)
+    C = np.stack(c)
+    for t in range(T):
+        assert np.all(lat[t] <= C[:t + 1].max(axis=0) + 1e-12) and np.all(lat[t] >= C[:t + 1].min(axis=0) - 1e-12)
+
+
+def test_mla_prefill_last_token_is_the_g1_decode_over_the_prompt():
+    # the last prompt token's output is a g = 1 decode of a sequence whose cache holds the prompt
+    rng = np.random.default_rng(5)
+    T, H, L, R, dv = 70, 3, 16, 4, 5
+    x = rng.standard_normal((T, L))
+    kpe = np.asarray(torch.from_numpy(rng.standard_normal((T, R))).to(torch.bfloat16).to(torch.float64))
+    q = rng.standard_normal((T, H, L))
+    q_pe = rng.standard_normal((T, H, R))
+    w = rng.standard_normal((H, L, dv))
+    out = ref.mla_prefill(x, kpe, q, q_pe, 0.2, transform=ref.TRANSFORM_HADAMARD, w_uv=w)
+    ckv = np.zeros((2, 1, 64, L)); kc = np.zeros((2, 64, R))
+    c = ref.bf16_round(ref.append_values(x, 1, ref.TRANSFORM_HADAMARD))[:, 0, :]
+    for t in range(T):
+        ckv[t // 64, 0, t % 64] = c[t]
+        kc[t // 64, t % 64] = kpe[t]
+    for t in (0, 63, 64, T - 1):
+        dec = ref.decode(q[t][None], q_pe[t][None], ckv, kc, np.array([[0, 1]]), np.array([t + 1]), 0.2,
+                         max_pages_per_seq=2, w_uv=w)
+        np.testing.assert_allclose(out[t], dec[0], rtol=1e-12, atol=1e-12)
