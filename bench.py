@@ -650,6 +650,64 @@ def config_of(spec, l2=None):
 
 # ---------------------------------------------------------------- main
 
+def run_prefill(args, rank):
+    """MLA-form prefill of one T-token prompt (DeepSeek-V3 shape, g = 2 cache for the decode that follows),
+    timed with CUDA events over K prefills after W warm-ups.  The work is the absorbed form's causal
+    attention: per query t and key i <= t, 2H(L+R) + 2HL FLOPs (scores and output over the whole latent),
+    plus the W_UV projection of every output row; the line reports prompt tokens per second and the
+    tensor-pipe roofline against the measured bf16 peak."""
+    if rank != 0:
+        return None
+    import torch
+    from latent_attention_decode_tpla_b200 import inputs as gen
+    from latent_attention_decode_tpla_b200 import prefill, tpla
+    T, H, L, R, dv, g = args.prefill, 128, 512, 64, 128, 2
+    gcpu = torch.Generator().manual_seed(0)
+    bf = lambda t: t.to(torch.bfloat16).cuda()
+    x, kpe = bf(torch.randn(T, L, generator=gcpu)), bf(torch.randn(T, R, generator=gcpu))
+    q, q_pe = bf(torch.randn(T, H, L, generator=gcpu)), bf(torch.randn(T, H, R, generator=gcpu))
+    w_uv = bf(torch.randn(H, L, dv, generator=gcpu) / math.sqrt(L))
+    maxp = (T + 63) // 64
+    dims = tpla.make_dims(B=1, H=H, L=L, R=R, dv=dv, g=g, max_pages_per_seq=maxp, num_pages=maxp,
+                          softmax_scale=1 / math.sqrt(192))
+    ckv = torch.zeros((maxp, g, 64, L // g), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((maxp, 64, R), dtype=torch.bfloat16, device="cuda")
+    row = torch.arange(maxp, dtype=torch.int32, device="cuda")
+    out = torch.empty((T, H, dv), dtype=torch.float32, device="cuda")
+    run = lambda: prefill.mla_prefill(dims, x, kpe, q, q_pe, w_uv, tpla.TRANSFORM_HADAMARD, None, None, 1e-6, row,
+                                      ckv, kc, out)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    if tpla.check_device_status() != tpla.TPLA_OK:
+        raise RuntimeError("device status after the prefill warm-up")
+    sampler = ClockSampler(0)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.start()
+    e0.record()
+    for _ in range(args.steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    pairs = T * (T + 1) // 2
+    flops = pairs * (2 * H * (L + R) + 2 * H * L) + T * 2 * H * L * dv
+    peaks, kind = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"metric": "MLA-form prefill prompt tokens/s", "value": T / (ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_prefill": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "mla_prefill_dsv3_%d" % T, "prompt": T, "heads": H, "kv_lora_rank": L,
+                       "rope_dim": R, "v_head_dim": dv, "decode_shards_g": g, "transform": "hadamard",
+                       "form": "absorbed MLA attention over the prompt (one-shard tcgen05 kernel), chunks of 64"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "peak_kind": kind,
+                         "flops_per_prefill": flops},
+            "clocks": clocks}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -667,6 +725,8 @@ def main():
                     help="tokens per tile of the tcgen05 kernel for L/g <= 256 (0: the library default)")
     ap.add_argument("--attn-replay-s", type=float, default=MIN_TIMED_S,
                     help="seconds the attention-only replays span at least (5 replays at least)")
+    ap.add_argument("--prefill", type=int, default=0,
+                    help="time the MLA-form prefill of a prompt of this many tokens instead of decode")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     spec = workload_spec(args.workload)
@@ -686,6 +746,11 @@ def main():
     if args.tile:
         from latent_attention_decode_tpla_b200 import tpla
         tpla.set_option(tpla.OPT_TILE_TOKENS, args.tile)
+    if args.prefill:
+        line = run_prefill(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     if args.tp:
         line = run_tp_arm(args, spec, rank, world, local)
         if line is not None:
