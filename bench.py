@@ -675,7 +675,7 @@ def run_prefill(args, rank):
     row = torch.arange(maxp, dtype=torch.int32, device="cuda")
     out = torch.empty((T, H, dv), dtype=torch.float32, device="cuda")
     run = lambda: prefill.mla_prefill(dims, x, kpe, q, q_pe, w_uv, tpla.TRANSFORM_HADAMARD, None, None, 1e-6, row,
-                                      ckv, kc, out)
+                                      ckv, kc, out, chunk=args.prefill_chunk)
     for _ in range(args.warmup):
         run()
     torch.cuda.synchronize()
@@ -701,7 +701,7 @@ def run_prefill(args, rank):
             "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "mla_prefill_dsv3_%d" % T, "prompt": T, "heads": H, "kv_lora_rank": L,
                        "rope_dim": R, "v_head_dim": dv, "decode_shards_g": g, "transform": "hadamard",
-                       "form": "absorbed MLA attention over the prompt (one-shard tcgen05 kernel), chunks of 64"},
+                       "form": "absorbed MLA attention over the prompt (one-shard tcgen05 kernel), chunks of %d" % args.prefill_chunk},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": None, "peak_kind": kind,
                          "flops_per_prefill": flops},
@@ -727,6 +727,7 @@ def main():
                     help="seconds the attention-only replays span at least (5 replays at least)")
     ap.add_argument("--prefill", type=int, default=0,
                     help="time the MLA-form prefill of a prompt of this many tokens instead of decode")
+    ap.add_argument("--prefill-chunk", type=int, default=64, help="prompt tokens per attention call of the prefill")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     spec = workload_spec(args.workload)
